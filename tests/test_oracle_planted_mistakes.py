@@ -1,0 +1,61 @@
+"""The oracle's pins must catch plausible mistakes (CPU only).
+
+Each case copies oracle/oracle.c, plants one mistake by a textual edit (a
+dropped term, a wrong sign, index, bias, rounding direction, transposed
+layout ...), compiles the copy and runs the oracle pin tests against it in a
+child process (FGFP8_ORACLE_LIB points the wrapper at the broken build).  The
+pins pass on the real oracle (the other test files) and must fail on every
+mutant.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "oracle.c")
+PIN_TESTS = ["tests/test_oracle_codec.py", "tests/test_oracle_quant.py", "tests/test_oracle_gemm.py"]
+
+MUTANTS = {
+    "tie_to_odd": ("pick = (lo % 2 == 0) ? lo : up;", "pick = (lo % 2 == 0) ? up : lo;"),
+    "truncate_not_round": ("if (dlo < dup) pick = lo;", "if (dlo < dup + 1e9) pick = lo;"),
+    "exponent_bias_8": ("mag = ldexp(1.0 + (double)m / 8.0, e - 7);",
+                        "mag = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    "subnormal_exponent": ("mag = ldexp((double)m / 8.0, -6);", "mag = ldexp((double)m / 8.0, -7);"),
+    "sign_dropped": ("uint8_t sign = signbit(v) ? 0x80 : 0x00;", "uint8_t sign = 0x00;"),
+    "scale_divisor_447": ("float orc_scale_f32(float amax_c) { return amax_c / 448.0f; }",
+                          "float orc_scale_f32(float amax_c) { return amax_c / 447.0f; }"),
+    "ue8m0_rounds_down": ("int p = (f == 0.5f) ? x - 1 : x;", "int p = x - 1;"),
+    "amax_floor_1e-3": ("#define ORC_AMAX_FLOOR 1e-4f", "#define ORC_AMAX_FLOOR 1e-3f"),
+    "act_scale_rows_reversed": ("((float*)Xs)[g * ld_s + m] = sf;",
+                                "((float*)Xs)[g * ld_s + (M - 1 - m)] = sf;"),
+    "weight_amax_first_row_only": ("float amax_c = amax_clamped(blk, ORC_GROUP, ldw, ORC_GROUP);",
+                                   "float amax_c = amax_clamped(blk, ORC_GROUP, ldw, 1);"),
+    "gemm_weight_scale_dropped": ("y += (sa * sw) * p;", "y += sa * p;"),
+    "gemm_weight_scale_transposed": (
+        "double sw = scale_at(Ws, ws_off + (n / ORC_GROUP) * KB + kb, fmt);",
+        "double sw = scale_at(Ws, ws_off + kb * NB + n / ORC_GROUP, fmt);"),
+    "gemm_abs_weight": ("double prod = table[xr[k]] * table[wr[k]];",
+                        "double prod = table[xr[k]] * fabs(table[wr[k]]);"),
+    "grouped_segment_boundary": ("if (offs[i] <= m && m < offs[i + 1]) { e = i; break; }",
+                                 "if (offs[i] <= m && m <= offs[i + 1]) { e = i; break; }"),
+}
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_reject_planted_mistake(tmp_path, name):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not found exactly once"
+    mutant_c = tmp_path / "oracle_mutant.c"
+    mutant_c.write_text(src.replace(old, new))
+    so = tmp_path / "liboracle_mutant.so"
+    subprocess.run(["gcc", "-std=c11", "-O2", "-ffp-contract=off", "-fopenmp", "-fPIC", "-shared",
+                    "-w", "-o", str(so), str(mutant_c), "-lm"], check=True)
+    env = dict(os.environ, FGFP8_ORACLE_LIB=str(so), OMP_NUM_THREADS="4")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider", *PIN_TESTS],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"mutant {name} passed every pin:\n{r.stdout[-2000:]}"
+    assert "failed" in r.stdout, r.stdout[-2000:] + r.stderr[-2000:]
