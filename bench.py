@@ -1,0 +1,516 @@
+#!/usr/bin/env python3
+"""Benchmark of the fine-grained FP8 W8A8 linear layer on B200.
+
+One step = one pass of the hot path over one batch of synthetic input:
+dynamic per-token 1x128 activation quantization (fgfp8_quant_act) followed by
+the block-scaled FP8 GEMM with its bf16 epilogue (fgfp8_gemm, or
+fgfp8_grouped_gemm for the MoE workload).  Weights are quantized once before
+timing (fgfp8_quant_weight, reported separately), as a deployed layer holds
+pre-quantized weights.
+
+Default workload: the Llama-3-8B attention projection in prefill,
+X [4096, 4096] x W [4096, 4096], fp32 block scales.  Other workloads can be
+chosen with --workload (see workloads/).
+
+Timing: W warm-up steps, then K timed steps.  L2 is flushed (a 256 MB write)
+before every step, outside the timed events.  Each kernel is bracketed by
+CUDA events on the launching stream.  For N > 1 (torchrun) every rank runs
+its own replica of the workload with no collective on the data path, and
+rank 0 reports the max over ranks.
+
+--impl reference runs the CPU oracle (the plain C implementation under
+oracle/) on the host cores: on each step it quantizes and multiplies a
+bounded sample of rows of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "block-scaled FP8 GEMM TFLOP/s (% FP8 peak); act-quant GB/s (% HBM)"
+L2_FLUSH_BYTES = 256 << 20
+FP8_OVER_BF16 = 2.0            # nominal dense fp8 / bf16 tensor ratio on B200 (4.5 / 2.25 PFLOP/s)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+WORKLOAD_ALIASES = {
+    "llama_attn": workloads.LLAMA_ATTN.name, "tiny": workloads.TINY.name,
+    "llama_gate_up": workloads.LLAMA_GATE_UP.name, "llama_down": workloads.LLAMA_DOWN.name,
+    **{f"ds_decode_m{m}": workloads.DS_DECODE[m].name for m in (1, 8, 32, 64)},
+    "moe": workloads.MOE.name,
+}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    return {**FALLBACK_PEAKS, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of the GPU's clocks and throttle reasons during the
+    timed region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            ids = subprocess.run(["nvidia-smi", "--query-gpu=index,uuid", "--format=csv,noheader"],
+                                 capture_output=True, text=True, timeout=20).stdout
+            self.index = None
+            for line in ids.strip().splitlines():
+                idx, u = [x.strip() for x in line.split(",")]
+                if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                    self.index = idx
+            if self.index is None:
+                self.index = str(device_index)
+        except Exception:
+            self.index = None
+
+    def start(self):
+        if self.index is None:
+            return
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.index, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path).read().strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[3:]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for _, _, flags in rows:
+            for n, v in zip(names[1:], flags[1:]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "samples": len(rows), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- workloads on the GPU
+class DenseLayer:
+    """X [M, K] bf16 and pre-quantized W for one dense linear layer."""
+
+    def __init__(self, cfg: workloads.Linear, dev):
+        import fine_grained_fp8_token_b200 as fg
+        self.fg, self.cfg, self.dev = fg, cfg, dev
+        self.X = workloads.activations((cfg.M, cfg.K), cfg.x_kind, cfg.seed, device=dev)
+        W = workloads.weights((cfg.N, cfg.K), cfg.seed + 1, device=dev)
+        sdt = torch.float32 if cfg.fmt == 0 else torch.uint8
+        self.W = W
+        self.Wq = torch.empty((cfg.N, cfg.K), dtype=torch.uint8, device=dev)
+        self.Ws = torch.empty((cfg.N // 128, cfg.K // 128), dtype=sdt, device=dev)
+        self.ld_s = fg.scale_rows(cfg.M, cfg.fmt)
+        self.Xq = torch.empty((cfg.M, cfg.K), dtype=torch.uint8, device=dev)
+        self.Xs = torch.empty((cfg.K // 128, self.ld_s), dtype=sdt, device=dev)
+        self.Y = torch.empty((cfg.M, cfg.N), dtype=torch.bfloat16, device=dev)
+        self.quant_weight()
+
+    def quant_weight(self):
+        self.fg.quant_weight(self.W, self.cfg.fmt, Wq=self.Wq, Ws=self.Ws)
+
+    def quant_act(self, X=None):
+        self.fg.quant_act(self.X if X is None else X, self.cfg.fmt, Xq=self.Xq, Xs=self.Xs, ld_s=self.ld_s)
+
+    def gemm(self):
+        self.fg.gemm(self.Xq, self.Xs, self.Wq, self.Ws, self.cfg.fmt, Y=self.Y)
+
+    def flops(self):
+        c = self.cfg
+        return 2.0 * c.M * c.N * c.K
+
+    def act_bytes(self):
+        c = self.cfg
+        return 2.0 * c.M * c.K + c.M * c.K + (4 if c.fmt == 0 else 1) * c.M * c.K / 128
+
+    def gemm_bytes(self):
+        c = self.cfg
+        sb = 4 if c.fmt == 0 else 1
+        return c.M * c.K + c.N * c.K + sb * (c.M * c.K / 128 + c.N * c.K / 16384) + 2.0 * c.M * c.N
+
+    def weight_bytes(self):
+        c = self.cfg
+        return 3.0 * c.N * c.K + (4 if c.fmt == 0 else 1) * c.N * c.K / 16384
+
+    def describe(self):
+        c = self.cfg
+        return {"workload": c.name, "M": c.M, "N": c.N, "K": c.K,
+                "scales": "fp32" if c.fmt == 0 else "ue8m0", "x": c.x_kind}
+
+    def host_io(self):
+        return self.X, self.Y
+
+
+class MoELayer:
+    """Grouped expert layer: routed token rows and pre-quantized experts."""
+
+    def __init__(self, cfg: workloads.MoE, dev):
+        import fine_grained_fp8_token_b200 as fg
+        self.fg, self.cfg, self.dev = fg, cfg, dev
+        self.r = workloads.moe_routing(cfg)
+        self.X = workloads.moe_grouped_rows(workloads.moe_tokens(cfg, device=dev), self.r)
+        sdt = torch.float32 if cfg.fmt == 0 else torch.uint8
+        self.Wq = torch.empty((cfg.E, cfg.N, cfg.K), dtype=torch.uint8, device=dev)
+        self.Ws = torch.empty((cfg.E, cfg.N // 128, cfg.K // 128), dtype=sdt, device=dev)
+        for e in range(cfg.E):
+            fg.quant_weight(workloads.moe_expert_weight(cfg, e, device=dev), cfg.fmt, Wq=self.Wq[e], Ws=self.Ws[e])
+        self.offs = torch.as_tensor(self.r.group_offs, device=dev)
+        M = self.r.M_total
+        self.ld_s = fg.scale_rows(M, cfg.fmt)
+        self.Xq = torch.empty((M, cfg.K), dtype=torch.uint8, device=dev)
+        self.Xs = torch.empty((cfg.K // 128, self.ld_s), dtype=sdt, device=dev)
+        self.Y = torch.empty((M, cfg.N), dtype=torch.bfloat16, device=dev)
+        self.W = workloads.moe_expert_weight(cfg, 0, device=dev)     # for timing the weight quantizer
+
+    def quant_weight(self):
+        self.fg.quant_weight(self.W, self.cfg.fmt, Wq=self.Wq[0], Ws=self.Ws[0])
+
+    def quant_act(self, X=None):
+        self.fg.quant_act(self.X if X is None else X, self.cfg.fmt, Xq=self.Xq, Xs=self.Xs, ld_s=self.ld_s)
+
+    def gemm(self):
+        self.fg.grouped_gemm(self.Xq, self.Xs, self.Wq, self.Ws, self.offs, self.cfg.fmt, Y=self.Y)
+
+    def flops(self):
+        c = self.cfg
+        return 2.0 * float(self.r.counts.sum()) * c.N * c.K      # useful rows only, no padding
+
+    def act_bytes(self):
+        c = self.cfg
+        M = self.r.M_total
+        return 3.0 * M * c.K + (4 if c.fmt == 0 else 1) * M * c.K / 128
+
+    def gemm_bytes(self):
+        c = self.cfg
+        M = self.r.M_total
+        sb = 4 if c.fmt == 0 else 1
+        return M * c.K + c.E * c.N * c.K + sb * (M * c.K / 128 + c.E * c.N * c.K / 16384) + 2.0 * M * c.N
+
+    def weight_bytes(self):
+        c = self.cfg
+        return 3.0 * c.N * c.K + (4 if c.fmt == 0 else 1) * c.N * c.K / 16384
+
+    def describe(self):
+        c = self.cfg
+        return {"workload": c.name, "experts": c.E, "N": c.N, "K": c.K, "tokens": c.tokens, "topk": c.topk,
+                "zipf": c.zipf, "M_total_padded": self.r.M_total, "rows_routed": int(self.r.counts.sum()),
+                "max_rows_per_expert": int(self.r.counts.max()), "scales": "fp32" if c.fmt == 0 else "ue8m0"}
+
+    def host_io(self):
+        return self.X, self.Y
+
+
+def make_layer(name, dev):
+    name = WORKLOAD_ALIASES.get(name, name)
+    if name == workloads.MOE.name:
+        return MoELayer(workloads.MOE, dev)
+    return DenseLayer(workloads.LINEARS[name], dev)
+
+
+# ---------------------------------------------------------------- timing
+def run_gpu(args, rank, world, dev):
+    layer = make_layer(args.workload, dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    launches_per_step = 2
+
+    def step():
+        layer.quant_act()
+        layer.gemm()
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    layer.fg.check_device_status()
+
+    n = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+    sampler = ClockSampler(dev.index)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    for i in range(n):
+        flush.fill_(1)
+        ev[i][0].record(stream)
+        layer.quant_act()
+        ev[i][1].record(stream)
+        layer.gemm()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    layer.fg.check_device_status()
+    quant_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(n)]
+    gemm_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(n)]
+    step_ms = [q + g for q, g in zip(quant_ms, gemm_ms)]
+    total_ms = sum(step_ms)
+
+    # weight quantization (offline step, reported, not part of the step)
+    wq_ms = []
+    for _ in range(max(3, min(n, 10))):
+        flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        layer.quant_weight()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        wq_ms.append(a.elapsed_time(b))
+
+    # end to end through the public API with host buffers: pinned X in,
+    # quantize + GEMM, pinned Y out, copies inside the timed events
+    X_dev, Y_dev = layer.host_io()
+    X_host = torch.empty(X_dev.shape, dtype=X_dev.dtype, pin_memory=True)
+    X_host.copy_(X_dev)
+    Y_host = torch.empty(Y_dev.shape, dtype=Y_dev.dtype, pin_memory=True)
+    X_stage = torch.empty_like(X_dev)
+    e2e_ms = []
+    e2e_steps = max(3, min(n, 10))
+    for i in range(e2e_steps + 2):
+        flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        X_stage.copy_(X_host, non_blocking=True)
+        layer.quant_act(X_stage)
+        layer.gemm()
+        Y_host.copy_(Y_dev, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        if i >= 2:
+            e2e_ms.append(a.elapsed_time(b))
+    h2d = X_host.numel() * X_host.element_size()
+    d2h = Y_host.numel() * Y_host.element_size()
+
+    stats = torch.tensor([total_ms, sum(gemm_ms), sum(quant_ms), statistics.mean(e2e_ms),
+                          statistics.mean(wq_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(stats, op=torch.distributed.ReduceOp.MAX)
+    total_ms, gemm_total, quant_total, e2e_mean, wq_mean = stats.tolist()
+    return layer, {"total_ms": total_ms, "gemm_ms": gemm_total / n, "quant_ms": quant_total / n,
+                   "e2e_ms": e2e_mean, "wq_ms": wq_mean, "clocks": clocks, "h2d": h2d, "d2h": d2h,
+                   "launches": launches_per_step * n}
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+class OracleSample:
+    """The oracle on a bounded sample of the workload: r rows of X quantized
+    and multiplied by the (pre-quantized, untimed) full weight."""
+
+    def __init__(self, name, rows):
+        import oracle
+        self.oracle = oracle
+        name = WORKLOAD_ALIASES.get(name, name)
+        if name == workloads.MOE.name:
+            cfg = workloads.MOE
+            r = workloads.moe_routing(cfg)
+            e = int(np.argmax(r.counts))                    # the busiest expert's rows
+            tok = r.row_token[r.group_offs[e]:r.group_offs[e] + r.counts[e]]
+            X = workloads.moe_tokens(cfg)[torch.as_tensor(tok[:rows])]
+            W = workloads.moe_expert_weight(cfg, e)
+            self.N, self.K, self.fmt = cfg.N, cfg.K, cfg.fmt
+            self.desc = f"{min(rows, len(tok))} routed rows of expert {e} x its [4096, 7168] weight"
+        else:
+            cfg = workloads.LINEARS[name]
+            X, W = workloads.linear_inputs(cfg)
+            X = X[:rows]
+            self.N, self.K, self.fmt = cfg.N, cfg.K, cfg.fmt
+            self.desc = f"first {min(rows, cfg.M)} of {cfg.M} rows x the full [{cfg.N}, {cfg.K}] weight"
+        self.X = X.contiguous().view(torch.int16).numpy().view(np.uint16)
+        self.Wq, self.Ws = oracle.quant_weight(W.contiguous().view(torch.int16).numpy().view(np.uint16), self.fmt)
+        self.rows = self.X.shape[0]
+
+    def step(self):
+        Xq, Xs = self.oracle.quant_act(self.X, self.fmt)
+        self.oracle.gemm(Xq, Xs, self.Wq, self.Ws, self.fmt)
+
+    def flops(self):
+        return 2.0 * self.rows * self.N * self.K
+
+
+def calibrated_sample(name, target_s):
+    """Grow the row sample until one oracle step takes about target_s."""
+    rows = 4
+    s = OracleSample(name, rows)
+    t0 = time.perf_counter()
+    s.step()
+    dt = max(time.perf_counter() - t0, 1e-3)
+    rows = max(1, int(rows * target_s / dt))
+    return OracleSample(name, rows)
+
+
+def cpu_baseline(name, target_s=15.0):
+    os.environ.setdefault("OMP_NUM_THREADS", str(cpu_cores()))
+    s = calibrated_sample(name, target_s / 3)
+    t0 = time.perf_counter()
+    reps = 0
+    while time.perf_counter() - t0 < target_s or reps == 0:
+        s.step()
+        reps += 1
+    dt = (time.perf_counter() - t0) / reps
+    return {"value": s.flops() / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"{s.desc}, fmt {'fp32' if s.fmt == 0 else 'ue8m0'}; quantize + GEMM per step, "
+                      f"{reps} steps of {dt:.2f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    os.environ.setdefault("OMP_NUM_THREADS", str(cpu_cores()))
+    s = calibrated_sample(args.workload, 2.0)
+    for _ in range(args.warmup):
+        s.step()
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        s.step()
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * statistics.mean(times)
+    value = s.flops() / (ms / 1e3) / 1e12
+    name = WORKLOAD_ALIASES.get(args.workload, args.workload)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": name, "sample_rows": s.rows, "parallelism": "host cores (OpenMP)"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+                             "sample": s.desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="fgfp8", choices=["fgfp8", "reference"])
+    ap.add_argument("--workload", default="llama_attn",
+                    help="one of: " + ", ".join(WORKLOAD_ALIASES))
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (quick runs)")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        return run_reference(args)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    layer, r = run_gpu(args, rank, world, dev)
+    peaks = measured_peaks()
+    n = args.steps
+    step_ms = r["total_ms"] / n
+    flops = layer.flops()
+    value = world * flops / (step_ms / 1e3) / 1e12
+    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+    gemm_tflops = flops / (r["gemm_ms"] / 1e3) / 1e12
+    gemm_gbs = layer.gemm_bytes() / (r["gemm_ms"] / 1e3) / 1e9
+    act_gbs = layer.act_bytes() / (r["quant_ms"] / 1e3) / 1e9
+    wq_gbs = layer.weight_bytes() / (r["wq_ms"] / 1e3) / 1e9
+    hbm_bound = gemm_tflops / fp8_peak < gemm_gbs / peaks["hbm_gbs"]
+    if hbm_bound:
+        roofline = {"bound": "hbm", "achieved": gemm_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": gemm_gbs / peaks["hbm_gbs"], "traffic": None,
+                    "kernel": "gemm_blockscaled_kernel",
+                    "peak_source": f"{peaks['source']} HBM copy bandwidth"}
+    else:
+        roofline = {"bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
+                    "frac": gemm_tflops / fp8_peak, "traffic": None, "kernel": "gemm_blockscaled_kernel",
+                    "peak_source": f"{peaks['source']} cuBLAS bf16 burst x {FP8_OVER_BF16:g} (nominal fp8/bf16)"}
+    line = {
+        "impl": "fgfp8", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": n,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3xe4m3->f32", "data": "synthetic (seeded, see workloads/)",
+        "config": {**layer.describe(), "l2": "flushed (256 MB write) before every timed step",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": roofline,
+        "kernels": {
+            "gemm": {"us": 1e3 * r["gemm_ms"], "tflops": gemm_tflops, "frac_fp8_peak": gemm_tflops / fp8_peak,
+                     "gbs": gemm_gbs, "frac_hbm": gemm_gbs / peaks["hbm_gbs"]},
+            "quant_act": {"us": 1e3 * r["quant_ms"], "gbs": act_gbs, "frac_hbm": act_gbs / peaks["hbm_gbs"],
+                          "bytes": layer.act_bytes()},
+            "quant_weight_offline": {"us": 1e3 * r["wq_ms"], "gbs": wq_gbs, "frac_hbm": wq_gbs / peaks["hbm_gbs"],
+                                     "bytes": layer.weight_bytes()},
+        },
+        "e2e": {"value": world * flops / (r["e2e_ms"] / 1e3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"], "ms_per_step": r["e2e_ms"]},
+        "gpu_launches": r["launches"],
+        "clocks": r["clocks"],
+        "peaks": peaks,
+    }
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

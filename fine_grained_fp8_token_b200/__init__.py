@@ -1,0 +1,175 @@
+"""Python binding of libfgfp8 — fine-grained FP8 W8A8 linear layers on B200.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library (include/fgfp8.h).  PyTorch supplies device memory and streams.  There
+is no CPU path: without the compiled library or without an sm_100a GPU every
+compute call raises.
+
+Raw entry points keep the C names (``fgfp8_quant_act`` ...) and take integers
+(device addresses, sizes, a stream handle).  The tensor helpers
+(``quant_act``, ``quant_weight``, ``gemm``, ``grouped_gemm``) allocate the
+outputs with torch on the input's device and call the raw entry points on the
+current stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+SCALE_F32 = 0
+SCALE_UE8M0 = 1
+
+_STATUS = {
+    0: "FGFP8_OK", 1: "FGFP8_ERR_INVALID_ARG", 2: "FGFP8_ERR_SHAPE", 3: "FGFP8_ERR_ALIGN",
+    4: "FGFP8_ERR_UNSUPPORTED", 5: "FGFP8_ERR_CUDA", 6: "FGFP8_ERR_TIMEOUT", 7: "FGFP8_ERR_DEVICE",
+}
+
+# Every symbol include/fgfp8.h declares, with (restype, argtypes).
+_P, _I64, _I32, _INT = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int
+SIGNATURES = {
+    "fgfp8_version": (_INT, []),
+    "fgfp8_last_error_string": (ctypes.c_char_p, []),
+    "fgfp8_quant_weight": (_INT, [_P, _I64, _I64, _I64, _P, _P, _INT, _P]),
+    "fgfp8_quant_act": (_INT, [_P, _I64, _I64, _I64, _P, _P, _I64, _INT, _P]),
+    "fgfp8_gemm": (_INT, [_P, _P, _I64, _P, _P, _P, _I64, _I64, _I64, _INT, _P]),
+    "fgfp8_grouped_gemm": (_INT, [_P, _P, _I64, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _INT, _P]),
+    "fgfp8_check_device_status": (_INT, [_P]),
+}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class FGFP8Error(RuntimeError):
+    def __init__(self, status: int, where: str, message: str):
+        self.status = status
+        super().__init__(f"{where}: {_STATUS.get(status, status)}: {message}")
+
+
+def library_path() -> str:
+    return os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfgfp8.so")
+
+
+def load(build_if_missing: bool = True) -> ctypes.CDLL:
+    """Load libfgfp8.so (building it with nvcc first when it is missing or
+    older than its sources).  Raises when the library cannot be produced."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            from . import build as _build
+            path = library_path()
+            if build_if_missing and _build.is_stale():
+                _build.build()
+            if not os.path.exists(path):
+                raise FGFP8Error(5, "load", f"{path} is missing; run fine_grained_fp8_token_b200.build")
+            lib = ctypes.CDLL(path)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        msg = load().fgfp8_last_error_string().decode(errors="replace")
+        raise FGFP8Error(status, where, msg)
+
+
+def _raw(name):
+    def call(*args):
+        return getattr(load(), name)(*args)
+    call.__name__ = name
+    return call
+
+
+fgfp8_version = _raw("fgfp8_version")
+fgfp8_quant_weight = _raw("fgfp8_quant_weight")
+fgfp8_quant_act = _raw("fgfp8_quant_act")
+fgfp8_gemm = _raw("fgfp8_gemm")
+fgfp8_grouped_gemm = _raw("fgfp8_grouped_gemm")
+fgfp8_check_device_status = _raw("fgfp8_check_device_status")
+
+
+def fgfp8_last_error_string() -> str:
+    return load().fgfp8_last_error_string().decode(errors="replace")
+
+
+# ---------------------------------------------------------------- tensor helpers
+def _stream(stream=None) -> int:
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def scale_rows(M: int, fmt: int) -> int:
+    """Padded row count (ld_s) of an activation scale array for M tokens."""
+    unit = 4 if fmt == SCALE_F32 else 16
+    return max(unit, (M + unit - 1) // unit * unit)
+
+
+def _scale_dtype(fmt: int):
+    import torch
+    return torch.float32 if fmt == SCALE_F32 else torch.uint8
+
+
+def quant_act(X, fmt: int, Xq=None, Xs=None, ld_s: int | None = None, stream=None):
+    """Per-token 1x128 quantization of X (bf16 [M, K], CUDA).  Returns
+    (Xq uint8 [M, K], Xs [K/128, ld_s]) with Xs[g, m] the scale of token m."""
+    import torch
+    M, K = X.shape
+    ld_s = scale_rows(M, fmt) if ld_s is None else ld_s
+    if Xq is None:
+        Xq = torch.empty((M, K), dtype=torch.uint8, device=X.device)
+    if Xs is None:
+        Xs = torch.empty((K // 128, ld_s), dtype=_scale_dtype(fmt), device=X.device)
+    _check(fgfp8_quant_act(X.data_ptr(), M, K, X.stride(0), Xq.data_ptr(), Xs.data_ptr(), ld_s, fmt,
+                           _stream(stream)), "fgfp8_quant_act")
+    return Xq, Xs
+
+
+def quant_weight(W, fmt: int, Wq=None, Ws=None, stream=None):
+    """128x128 block quantization of W (bf16 [N, K], CUDA).  Returns
+    (Wq uint8 [N, K], Ws [N/128, K/128])."""
+    import torch
+    N, K = W.shape
+    if Wq is None:
+        Wq = torch.empty((N, K), dtype=torch.uint8, device=W.device)
+    if Ws is None:
+        Ws = torch.empty((N // 128, K // 128), dtype=_scale_dtype(fmt), device=W.device)
+    _check(fgfp8_quant_weight(W.data_ptr(), N, K, W.stride(0), Wq.data_ptr(), Ws.data_ptr(), fmt,
+                              _stream(stream)), "fgfp8_quant_weight")
+    return Wq, Ws
+
+
+def gemm(Xq, Xs, Wq, Ws, fmt: int, Y=None, stream=None):
+    """Y = X W^T (bf16 [M, N]) from the quantized operands."""
+    import torch
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=Xq.device)
+    _check(fgfp8_gemm(Xq.data_ptr(), Xs.data_ptr(), Xs.shape[1], Wq.data_ptr(), Ws.data_ptr(), Y.data_ptr(),
+                      M, N, K, fmt, _stream(stream)), "fgfp8_gemm")
+    return Y
+
+
+def grouped_gemm(Xq, Xs, Wq, Ws, group_offs, fmt: int, Y=None, stream=None):
+    """M-grouped expert GEMM: Wq [E, N, K], Ws [E, N/128, K/128], group_offs
+    int32 [E+1] on the device.  Returns Y bf16 [M_total, N]."""
+    import torch
+    M_total, K = Xq.shape
+    E, N, _ = Wq.shape
+    if Y is None:
+        Y = torch.empty((M_total, N), dtype=torch.bfloat16, device=Xq.device)
+    _check(fgfp8_grouped_gemm(Xq.data_ptr(), Xs.data_ptr(), Xs.shape[1], Wq.data_ptr(), Ws.data_ptr(),
+                              Y.data_ptr(), group_offs.data_ptr(), E, M_total, N, K, fmt, _stream(stream)),
+           "fgfp8_grouped_gemm")
+    return Y
+
+
+def check_device_status(stream=None) -> None:
+    """Synchronize and raise if a kernel recorded a timeout or bad input."""
+    _check(fgfp8_check_device_status(_stream(stream)), "fgfp8_check_device_status")

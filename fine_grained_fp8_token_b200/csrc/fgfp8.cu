@@ -1,0 +1,330 @@
+// C ABI of the fine-grained FP8 W8A8 library (declared in include/fgfp8.h):
+// host-side validation, TMA descriptor encoding and kernel launches.  All
+// kernels live in this translation unit so that they share the device status
+// word without relocatable device code.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+#include <set>
+#include <utility>
+#include <string>
+
+#include "fgfp8.h"
+#include "gemm.cuh"
+#include "ptx.cuh"
+#include "quant.cuh"
+
+namespace {
+
+thread_local std::string t_last_error;
+
+fgfp8_status fail(fgfp8_status code, const std::string& msg) {
+  t_last_error = msg;
+  return code;
+}
+
+fgfp8_status ok() {
+  t_last_error.clear();
+  return FGFP8_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+fgfp8_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(FGFP8_ERR_CUDA, std::string(what) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")");
+}
+
+struct DeviceInfo {
+  int sm_count = 0;
+  int cc_major = 0, cc_minor = 0;
+};
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::once_flag g_dev_once[kMaxDevices];
+
+fgfp8_status current_device(int* dev_out, DeviceInfo* info) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(FGFP8_ERR_CUDA, "device index out of range");
+  std::call_once(g_dev_once[dev], [dev] {
+    cudaDeviceGetAttribute(&g_dev[dev].sm_count, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&g_dev[dev].cc_major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&g_dev[dev].cc_minor, cudaDevAttrComputeCapabilityMinor, dev);
+  });
+  *info = g_dev[dev];
+  *dev_out = dev;
+  if (info->cc_major != 10 || info->cc_minor != 0)
+    return fail(FGFP8_ERR_CUDA, "this library is built for sm_100a (B200); device " + std::to_string(dev) +
+                                    " has compute capability " + std::to_string(info->cc_major) + "." +
+                                    std::to_string(info->cc_minor));
+  return FGFP8_OK;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// 2-D map over a row-major u8 matrix [rows, cols] (row stride ld bytes) with a
+// box of 128 columns (one 128-byte swizzle row) by box_rows rows.
+fgfp8_status make_map_u8_sw128(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
+                               uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(FGFP8_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FGFP8_ERR_CUDA, "cuTensorMapEncodeTiled failed with code " + std::to_string(r));
+  return FGFP8_OK;
+}
+
+// Raise the dynamic shared-memory limit of a kernel, once per (kernel, device).
+fgfp8_status set_smem(const void* kernel, size_t bytes, int dev) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count({kernel, dev})) return FGFP8_OK;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  done.insert({kernel, dev});
+  return FGFP8_OK;
+}
+
+fgfp8_status check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return ok();
+}
+
+fgfp8_status check_fmt(int fmt) {
+  if (fmt != FGFP8_SCALE_F32 && fmt != FGFP8_SCALE_UE8M0)
+    return fail(FGFP8_ERR_INVALID_ARG, "fmt must be FGFP8_SCALE_F32 (0) or FGFP8_SCALE_UE8M0 (1)");
+  return FGFP8_OK;
+}
+
+fgfp8_status check_act_scales(const void* Xs, int64_t ld_s, int64_t M, int fmt) {
+  if (!Xs) return fail(FGFP8_ERR_INVALID_ARG, "Xs is NULL");
+  if (ld_s < M) return fail(FGFP8_ERR_SHAPE, "ld_s must be >= M");
+  if (ld_s >= (int64_t(1) << 31)) return fail(FGFP8_ERR_SHAPE, "ld_s must be < 2^31");
+  const int64_t unit = (fmt == FGFP8_SCALE_F32) ? 4 : 16;
+  if (ld_s % unit != 0)
+    return fail(FGFP8_ERR_ALIGN, fmt == FGFP8_SCALE_F32 ? "ld_s must be a multiple of 4 for fp32 scales"
+                                                        : "ld_s must be a multiple of 16 for UE8M0 scales");
+  if (!aligned(Xs, 16)) return fail(FGFP8_ERR_ALIGN, "Xs must be 16-byte aligned");
+  return FGFP8_OK;
+}
+
+// Launch one GEMM instantiation.
+template <int BN, int FMT, bool kGrouped>
+fgfp8_status launch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
+                         void* Y, int64_t M, int64_t N, int64_t K, const int32_t* offs, int E, int64_t b_rows,
+                         cudaStream_t stream, int dev) {
+  using C = fgfp8::GemmCfg<BN>;
+  CUtensorMap mA, mB;
+  fgfp8_status st = make_map_u8_sw128(&mA, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
+                                      static_cast<uint64_t>(K), 128);
+  if (st != FGFP8_OK) return st;
+  st = make_map_u8_sw128(&mB, Wq, static_cast<uint64_t>(b_rows), static_cast<uint64_t>(K), static_cast<uint64_t>(K),
+                         BN);
+  if (st != FGFP8_OK) return st;
+  auto kernel = fgfp8::gemm_blockscaled_kernel<BN, FMT, kGrouped>;
+  st = set_smem(reinterpret_cast<const void*>(kernel), C::kSmemBytes, dev);
+  if (st != FGFP8_OK) return st;
+  const int64_t tiles = ((M + C::kBM - 1) / C::kBM) * (N / BN);
+  if (tiles == 0) return ok();
+  kernel<<<static_cast<unsigned>(tiles), C::kThreads, C::kSmemBytes, stream>>>(
+      mA, mB, Xs, static_cast<uint32_t>(ld_s), Ws, reinterpret_cast<__nv_bfloat16*>(Y), static_cast<int>(M),
+      static_cast<int>(N), static_cast<int>(K), offs, E);
+  return check_launch("gemm launch");
+}
+
+template <bool kGrouped>
+fgfp8_status dispatch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws, void* Y,
+                           int64_t M, int64_t N, int64_t K, int fmt, const int32_t* offs, int E, int64_t b_rows,
+                           cudaStream_t s, int dev) {
+  // 256-wide tiles halve the promotion work per MMA; 128-wide ones when N is
+  // not a multiple of 256 or when there are few rows (more CTAs in flight).
+  const bool wide = (N % 256 == 0) && M > 128;
+  if (fmt == FGFP8_SCALE_F32) {
+    return wide ? launch_gemm<256, 0, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev)
+                : launch_gemm<128, 0, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev);
+  }
+  return wide ? launch_gemm<256, 1, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev)
+              : launch_gemm<128, 1, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev);
+}
+
+fgfp8_status check_gemm_common(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
+                               void* Y, int64_t M, int64_t N, int64_t K, int fmt) {
+  fgfp8_status st = check_fmt(fmt);
+  if (st != FGFP8_OK) return st;
+  if (M < 0 || N < 0 || K < 0) return fail(FGFP8_ERR_INVALID_ARG, "negative size");
+  if (K == 0 || K % 128 != 0) return fail(FGFP8_ERR_SHAPE, "K must be a positive multiple of 128");
+  if (N == 0 || N % 128 != 0) return fail(FGFP8_ERR_SHAPE, "N must be a positive multiple of 128");
+  if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+    return fail(FGFP8_ERR_SHAPE, "M, N and K must be < 2^31");
+  if (!Xq || !Wq || !Ws || !Y) return fail(FGFP8_ERR_INVALID_ARG, "a required pointer is NULL");
+  st = check_act_scales(Xs, ld_s, M, fmt);
+  if (st != FGFP8_OK) return st;
+  if (!aligned(Xq, 16) || !aligned(Wq, 16) || !aligned(Y, 16))
+    return fail(FGFP8_ERR_ALIGN, "Xq, Wq and Y must be 16-byte aligned");
+  if (fmt == FGFP8_SCALE_F32 && !aligned(Ws, 4)) return fail(FGFP8_ERR_ALIGN, "fp32 Ws must be 4-byte aligned");
+  return FGFP8_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fgfp8_version(void) { return FGFP8_VERSION; }
+
+const char* fgfp8_last_error_string(void) { return t_last_error.c_str(); }
+
+fgfp8_status fgfp8_quant_act(const void* X, int64_t M, int64_t K, int64_t ldx, uint8_t* Xq, void* Xs, int64_t ld_s,
+                             int fmt, void* stream) {
+  fgfp8_status st = check_fmt(fmt);
+  if (st != FGFP8_OK) return st;
+  if (M < 0 || K < 0 || ldx < 0) return fail(FGFP8_ERR_INVALID_ARG, "negative size");
+  if (K == 0 || K % 128 != 0) return fail(FGFP8_ERR_SHAPE, "K must be a positive multiple of 128");
+  if (ldx < K) return fail(FGFP8_ERR_SHAPE, "ldx must be >= K");
+  if (M == 0) return ok();
+  if (M * (K / 128) >= (int64_t(1) << 32) || K >= (int64_t(1) << 31))
+    return fail(FGFP8_ERR_SHAPE, "M*K/128 must be < 2^32 and K < 2^31");
+  if (!X || !Xq) return fail(FGFP8_ERR_INVALID_ARG, "X or Xq is NULL");
+  st = check_act_scales(Xs, ld_s, M, fmt);
+  if (st != FGFP8_OK) return st;
+  if (!aligned(X, 16) || ldx % 8 != 0) return fail(FGFP8_ERR_ALIGN, "X must be 16-byte aligned with ldx % 8 == 0");
+  if (!aligned(Xq, 16)) return fail(FGFP8_ERR_ALIGN, "Xq must be 16-byte aligned");
+  int dev;
+  DeviceInfo info;
+  st = current_device(&dev, &info);
+  if (st != FGFP8_OK) return st;
+
+  constexpr int kUnroll = 2;
+  const uint64_t groups = static_cast<uint64_t>(M) * (K / 128);
+  const uint64_t want = (groups * 16 + 256 * kUnroll - 1) / (256 * kUnroll);
+  const uint64_t cap = static_cast<uint64_t>(info.sm_count) * 8;
+  const unsigned blocks = static_cast<unsigned>(want < cap ? (want ? want : 1) : cap);
+  fgfp8::FastDiv kbd(static_cast<uint32_t>(K / 128));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (fmt == FGFP8_SCALE_F32)
+    fgfp8::quant_act_kernel<0, kUnroll><<<blocks, 256, 0, s>>>(reinterpret_cast<const uint16_t*>(X),
+                                                               static_cast<uint32_t>(M), static_cast<uint32_t>(K),
+                                                               static_cast<uint64_t>(ldx), Xq, Xs,
+                                                               static_cast<uint64_t>(ld_s), kbd);
+  else
+    fgfp8::quant_act_kernel<1, kUnroll><<<blocks, 256, 0, s>>>(reinterpret_cast<const uint16_t*>(X),
+                                                               static_cast<uint32_t>(M), static_cast<uint32_t>(K),
+                                                               static_cast<uint64_t>(ldx), Xq, Xs,
+                                                               static_cast<uint64_t>(ld_s), kbd);
+  return check_launch("quant_act launch");
+}
+
+fgfp8_status fgfp8_quant_weight(const void* W, int64_t N, int64_t K, int64_t ldw, uint8_t* Wq, void* Ws, int fmt,
+                                void* stream) {
+  fgfp8_status st = check_fmt(fmt);
+  if (st != FGFP8_OK) return st;
+  if (N < 0 || K < 0 || ldw < 0) return fail(FGFP8_ERR_INVALID_ARG, "negative size");
+  if (K == 0 || K % 128 != 0) return fail(FGFP8_ERR_SHAPE, "K must be a positive multiple of 128");
+  if (N % 128 != 0) return fail(FGFP8_ERR_SHAPE, "N must be a multiple of 128");
+  if (ldw < K) return fail(FGFP8_ERR_SHAPE, "ldw must be >= K");
+  if (N == 0) return ok();
+  if ((N / 128) * (K / 128) >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+    return fail(FGFP8_ERR_SHAPE, "(N/128)*(K/128) must be < 2^31");
+  if (!W || !Wq || !Ws) return fail(FGFP8_ERR_INVALID_ARG, "W, Wq or Ws is NULL");
+  if (!aligned(W, 16) || ldw % 8 != 0) return fail(FGFP8_ERR_ALIGN, "W must be 16-byte aligned with ldw % 8 == 0");
+  if (!aligned(Wq, 16)) return fail(FGFP8_ERR_ALIGN, "Wq must be 16-byte aligned");
+  if (fmt == FGFP8_SCALE_F32 && !aligned(Ws, 4)) return fail(FGFP8_ERR_ALIGN, "fp32 Ws must be 4-byte aligned");
+  int dev;
+  DeviceInfo info;
+  st = current_device(&dev, &info);
+  if (st != FGFP8_OK) return st;
+  const unsigned blocks = static_cast<unsigned>((N / 128) * (K / 128));
+  fgfp8::FastDiv kbd(static_cast<uint32_t>(K / 128));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (fmt == FGFP8_SCALE_F32)
+    fgfp8::quant_weight_kernel<0><<<blocks, 256, 0, s>>>(reinterpret_cast<const uint16_t*>(W),
+                                                         static_cast<uint32_t>(K), static_cast<uint64_t>(ldw), Wq, Ws,
+                                                         kbd);
+  else
+    fgfp8::quant_weight_kernel<1><<<blocks, 256, 0, s>>>(reinterpret_cast<const uint16_t*>(W),
+                                                         static_cast<uint32_t>(K), static_cast<uint64_t>(ldw), Wq, Ws,
+                                                         kbd);
+  return check_launch("quant_weight launch");
+}
+
+fgfp8_status fgfp8_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws, void* Y,
+                        int64_t M, int64_t N, int64_t K, int fmt, void* stream) {
+  if (M == 0 && fmt >= 0 && fmt <= 1 && N >= 0 && K >= 0) return ok();
+  fgfp8_status st = check_gemm_common(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, fmt);
+  if (st != FGFP8_OK) return st;
+  int dev;
+  DeviceInfo info;
+  st = current_device(&dev, &info);
+  if (st != FGFP8_OK) return st;
+  return dispatch_gemm<false>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, fmt, nullptr, 1, N,
+                              reinterpret_cast<cudaStream_t>(stream), dev);
+}
+
+fgfp8_status fgfp8_grouped_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
+                                void* Y, const int32_t* group_offs, int32_t E, int64_t M_total, int64_t N, int64_t K,
+                                int fmt, void* stream) {
+  if (E <= 0) return fail(FGFP8_ERR_INVALID_ARG, "E must be >= 1");
+  if (M_total % 128 != 0) return fail(FGFP8_ERR_SHAPE, "M_total must be a multiple of 128");
+  if (M_total == 0 && fmt >= 0 && fmt <= 1 && N >= 0 && K >= 0) return ok();
+  fgfp8_status st = check_gemm_common(Xq, Xs, ld_s, Wq, Ws, Y, M_total, N, K, fmt);
+  if (st != FGFP8_OK) return st;
+  if (!group_offs) return fail(FGFP8_ERR_INVALID_ARG, "group_offs is NULL");
+  if (!aligned(group_offs, 4)) return fail(FGFP8_ERR_ALIGN, "group_offs must be 4-byte aligned");
+  if (static_cast<int64_t>(E) * N >= (int64_t(1) << 31))
+    return fail(FGFP8_ERR_SHAPE, "E*N must be < 2^31");
+  int dev;
+  DeviceInfo info;
+  st = current_device(&dev, &info);
+  if (st != FGFP8_OK) return st;
+  return dispatch_gemm<true>(Xq, Xs, ld_s, Wq, Ws, Y, M_total, N, K, fmt, group_offs, E,
+                             static_cast<int64_t>(E) * N, reinterpret_cast<cudaStream_t>(stream), dev);
+}
+
+fgfp8_status fgfp8_check_device_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, fgfp8::g_device_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+  if (v == fgfp8::kDevOk) return ok();
+  const int zero = 0;
+  e = cudaMemcpyToSymbol(fgfp8::g_device_status, &zero, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
+  switch (v) {
+    case fgfp8::kDevTimeoutProducer:
+      return fail(FGFP8_ERR_TIMEOUT, "a GEMM producer wait exceeded its limit");
+    case fgfp8::kDevTimeoutMma:
+      return fail(FGFP8_ERR_TIMEOUT, "a GEMM MMA wait exceeded its limit");
+    case fgfp8::kDevTimeoutEpilogue:
+      return fail(FGFP8_ERR_TIMEOUT, "a GEMM epilogue wait exceeded its limit");
+    case fgfp8::kDevBadGroupOffsets:
+      return fail(FGFP8_ERR_DEVICE, "group_offs is inconsistent (not a non-decreasing 0..M_total cover)");
+    default:
+      return fail(FGFP8_ERR_DEVICE, "unknown device status " + std::to_string(v));
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,218 @@
+// Dynamic per-token (1x128) activation quantization and 128x128 block weight
+// quantization to FP8 E4M3 with fp32 or UE8M0 scales.
+//
+// Method ("Fine-grained FP8", introduction and "UE8M0 scale format"; E4M3
+// range from "FP8 W8A8", "Two FP8 representations"):
+//   amax  = max |x| over the group or block (NaN propagates), raised to 1e-4
+//   fp32  : s = amax / 448 (IEEE division), code = E4M3_rne_satfinite(x / s)
+//   UE8M0 : s = 2^ceil(log2(amax / 448)), stored as its biased exponent byte
+//
+// x / s is evaluated without a per-element division: with r = RN(1/s),
+// q0 = RN(|x| r), e = fma(-q0, s, |x|), q = fma(e, r, q0) is the correctly
+// rounded quotient (Markstein's theorem, "IA-64 and Elementary Functions",
+// 2000; Muller et al., "Handbook of Floating-Point Arithmetic", the FMA-based
+// division section).  A host-side test checks it against IEEE division on
+// every (bf16 element, bf16 amax) pair the kernel can meet.  For UE8M0 the
+// quotient is |x| * 2^-p, exact.  The sign of x is applied to the E4M3 code
+// afterwards, so -0 and tiny negatives keep it.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cstdint>
+
+namespace fgfp8 {
+
+constexpr int kGroup = 128;
+
+// Unsigned 32-bit division by a runtime-invariant divisor, by multiplication
+// (Granlund & Montgomery, "Division by invariant integers using
+// multiplication", PLDI 1994, the round-up variant for N = 32).
+struct FastDiv {
+  uint32_t d, mult, sh1, sh2;
+  __host__ __device__ explicit FastDiv(uint32_t divisor) : d(divisor) {
+    uint32_t l = 0;
+    while ((1ull << l) < divisor) ++l;                      // l = ceil(log2 d)
+    mult = static_cast<uint32_t>(((1ull << 32) * ((1ull << l) - divisor)) / divisor + 1);
+    sh1 = l < 1 ? l : 1;
+    sh2 = l > 1 ? l - 1 : 0;
+  }
+  __host__ __device__ __forceinline__ uint32_t div(uint32_t n) const {
+#ifdef __CUDA_ARCH__
+    const uint32_t t = __umulhi(mult, n);
+#else
+    const uint32_t t = static_cast<uint32_t>((static_cast<uint64_t>(mult) * n) >> 32);
+#endif
+    return (t + ((n - t) >> sh1)) >> sh2;
+  }
+};
+
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// max |x| bits over 8 packed bf16 (sign masked; NaN patterns compare above
+// every finite value and infinity, so they propagate).
+__device__ __forceinline__ uint32_t absmax_bits8(const uint4& v) {
+  const uint32_t m = 0x7FFF7FFFu;
+  uint32_t a = __vmaxu2(__vmaxu2(v.x & m, v.y & m), __vmaxu2(v.z & m, v.w & m));
+  return max(a & 0xFFFFu, a >> 16);
+}
+
+struct GroupScale {
+  float s;        // the scale (fp32 path) or 2^p (UE8M0 path)
+  float r;        // RN(1/s) (fp32 path) or the exact 2^-p (UE8M0 path)
+  uint32_t e8;    // UE8M0 byte
+};
+
+template <int FMT>
+__device__ __forceinline__ GroupScale make_scale(uint32_t amax_bits) {
+  float amax = __uint_as_float(amax_bits << 16);
+  float amax_c = amax < 1e-4f ? 1e-4f : amax;          // NaN stays NaN
+  float t = __fdiv_rn(amax_c, 448.0f);
+  GroupScale g;
+  if (FMT == 0) {
+    g.s = t;
+    g.r = __frcp_rn(t);
+    g.e8 = 0;
+  } else {
+    uint32_t b = __float_as_uint(t);
+    uint32_t e = b >> 23;                                // t > 0: sign bit clear
+    if ((b & 0x7FFFFFu) != 0u && e < 255u) e += 1u;      // round up to a power of two
+    g.e8 = e;
+    g.s = 0.0f;
+    g.r = (e >= 1u && e <= 253u) ? __uint_as_float((254u - e) << 23) : 0.0f;   // 2^(127-e)
+  }
+  return g;
+}
+
+// |x|/s for the magnitude bits `h` (bf16 without sign) of one element.
+template <int FMT>
+__device__ __forceinline__ float quotient(uint32_t h, const GroupScale& g) {
+  float a = __uint_as_float(h << 16);
+  if (FMT == 0) {
+    float q0 = __fmul_rn(a, g.r);
+    float e = __fmaf_rn(-q0, g.s, a);
+    return __fmaf_rn(e, g.r, q0);
+  } else {
+    return __fmul_rn(a, g.r);
+  }
+}
+
+// Two packed bf16 (w) -> two E4M3 codes in the low 16 bits (element 0 low).
+template <int FMT>
+__device__ __forceinline__ uint32_t quant_pair(uint32_t w, const GroupScale& g) {
+  float q_lo = quotient<FMT>(w & 0x7FFFu, g);
+  float q_hi = quotient<FMT>((w >> 16) & 0x7FFFu, g);
+  uint32_t c = __nv_cvt_float2_to_fp8x2(make_float2(q_lo, q_hi), __NV_SATFINITE, __NV_E4M3);
+  return (c & 0xFFFFu) | ((w >> 8) & 0x80u) | ((w >> 16) & 0x8000u);
+}
+
+template <int FMT>
+__device__ __forceinline__ uint2 quant8(const uint4& v, const GroupScale& g) {
+  uint2 out;
+  out.x = quant_pair<FMT>(v.x, g) | (quant_pair<FMT>(v.y, g) << 16);
+  out.y = quant_pair<FMT>(v.z, g) | (quant_pair<FMT>(v.w, g) << 16);
+  return out;
+}
+
+// ---------------------------------------------------------------------------
+// Activation quantization.  One half-warp per 128-element group (16 lanes x
+// 16 bytes), UNROLL groups in flight per half-warp, grid-stride over the
+// M*K/128 groups in row-major order.
+// X bf16 [M, K] row stride ldx  ->  Xq u8 [M, K] row stride K,
+// scales Xs[g * ld_s + m] (fp32 or UE8M0 byte).
+// ---------------------------------------------------------------------------
+template <int FMT, int UNROLL>
+__global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restrict__ X, uint32_t M, uint32_t K,
+                                                        uint64_t ldx, uint8_t* __restrict__ Xq,
+                                                        void* __restrict__ Xs, uint64_t ld_s, FastDiv kb_div) {
+  const uint32_t total = M * kb_div.d;
+  const uint32_t lane = threadIdx.x & 31u;
+  const uint32_t sub = lane & 15u;
+  const uint32_t hmask = 0xFFFFu << (lane & 16u);
+  const uint32_t hw = (blockIdx.x * blockDim.x + threadIdx.x) >> 4;
+  const uint32_t nhw = (gridDim.x * blockDim.x) >> 4;
+
+  for (uint32_t base = hw; base < total; base += nhw * UNROLL) {
+    uint4 v[UNROLL];
+    uint32_t m[UNROLL], g[UNROLL];
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const uint32_t gi = base + u * nhw;
+      if (gi < total) {
+        m[u] = kb_div.div(gi);
+        g[u] = gi - m[u] * kb_div.d;
+        v[u] = ld_stream_v4(X + m[u] * ldx + g[u] * kGroup + sub * 8u);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const uint32_t gi = base + u * nhw;
+      if (gi < total) {
+        uint32_t a = absmax_bits8(v[u]);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) a = max(a, __shfl_xor_sync(hmask, a, o));
+        const GroupScale gs = make_scale<FMT>(a);
+        const uint2 codes = quant8<FMT>(v[u], gs);
+        *reinterpret_cast<uint2*>(Xq + static_cast<uint64_t>(m[u]) * K + g[u] * kGroup + sub * 8u) = codes;
+        if (sub == 0) {
+          const uint64_t si = static_cast<uint64_t>(g[u]) * ld_s + m[u];
+          if (FMT == 0) reinterpret_cast<float*>(Xs)[si] = gs.s;
+          else reinterpret_cast<uint8_t*>(Xs)[si] = static_cast<uint8_t>(gs.e8);
+        }
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Weight quantization.  One 256-thread CTA per 128x128 block: half-warp h
+// owns rows h, h+16, ..., h+112 of the block; every thread keeps its eight
+// 16-byte chunks in registers across the block-wide amax reduction.
+// W bf16 [N, K] row stride ldw -> Wq u8 [N, K] row stride K,
+// Ws[nb * KB + kb] (row-major [N/128, K/128]).
+// ---------------------------------------------------------------------------
+template <int FMT>
+__global__ void __launch_bounds__(256) quant_weight_kernel(const uint16_t* __restrict__ W, uint32_t K,
+                                                           uint64_t ldw, uint8_t* __restrict__ Wq,
+                                                           void* __restrict__ Ws, FastDiv kb_div) {
+  __shared__ uint32_t s_max[8];
+  const uint32_t blk = blockIdx.x;
+  const uint32_t nb = kb_div.div(blk);
+  const uint32_t kb = blk - nb * kb_div.d;
+  const uint32_t t = threadIdx.x;
+  const uint32_t h = t >> 4, sub = t & 15u;
+  const uint64_t row0 = static_cast<uint64_t>(nb) * kGroup;
+  const uint32_t col = kb * kGroup + sub * 8u;
+
+  uint4 v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = ld_stream_v4(W + (row0 + h + 16u * i) * ldw + col);
+  uint32_t a = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a = max(a, absmax_bits8(v[i]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = max(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+  if ((t & 31u) == 0) s_max[t >> 5] = a;
+  __syncthreads();
+  a = s_max[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) a = max(a, s_max[i]);
+
+  const GroupScale gs = make_scale<FMT>(a);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint2 codes = quant8<FMT>(v[i], gs);
+    *reinterpret_cast<uint2*>(Wq + (row0 + h + 16u * i) * K + col) = codes;
+  }
+  if (t == 0) {
+    if (FMT == 0) reinterpret_cast<float*>(Ws)[blk] = gs.s;
+    else reinterpret_cast<uint8_t*>(Ws)[blk] = static_cast<uint8_t>(gs.e8);
+  }
+}
+
+}  // namespace fgfp8

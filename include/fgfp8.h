@@ -1,0 +1,151 @@
+/*
+ * fgfp8 — fine-grained FP8 W8A8 linear layers for NVIDIA B200 (sm_100a).
+ *
+ * C ABI.  Plain pointers and sizes only.  Every pointer argument is a DEVICE
+ * pointer on the current CUDA device, except where a comment says otherwise.
+ * `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ * stream).  The caller allocates and owns every buffer.  These calls never
+ * allocate device memory.
+ *
+ * Every call validates its arguments on the host first.  A violation returns
+ * an error code, launches nothing and leaves a message for
+ * fgfp8_last_error_string().  A call that passes validation enqueues its kernels
+ * on `stream` and returns FGFP8_OK without waiting for them.  There is no CPU
+ * fallback: on a machine without a usable sm_100a GPU every compute call
+ * returns FGFP8_ERR_CUDA.
+ *
+ * Method (page titles and sections of the source documentation):
+ *   - "Fine-grained FP8" (Transformers docs), introduction: weights are
+ *     quantized to 8 bits per 128x128 block; activations per token, in groups
+ *     that match the weight's 128-wide input-channel block.
+ *   - "Fine-grained FP8", "DeepGEMM fast path": the dynamic activation scheme
+ *     (scales computed from each group at run time).
+ *   - "Fine-grained FP8", "UE8M0 scale format": scales stored either as
+ *     float32 or as packed float8_e8m0fnu (a power of two 2^(e-127) in one
+ *     byte).
+ *   - "FP8 W8A8" (vLLM docs), "Two FP8 representations": E4M3 has one sign,
+ *     four exponent and three mantissa bits, reaches +-448, and has NaN.
+ * The steps the pages leave open are fixed as follows.  Each step is one
+ * IEEE fp32 operation with round-to-nearest-even:
+ *   amax   = max |x| over the group/block; it is raised to 1e-4 if smaller,
+ *            and a NaN element makes it NaN
+ *   fp32   : scale = amax / 448
+ *   UE8M0  : scale = the smallest power of two >= amax / 448
+ *   code   = E4M3( x / scale ), rounded to nearest even and saturated to +-448
+ *   GEMM   : Y[m,n] = bf16_rne( sum_kb sa[m,kb] * sw[n/128,kb] *
+ *                               sum_{k in block kb} Xq[m,k] * Wq[n,k] ).
+ * The GEMM accumulates in fp32.  Its result is accurate to within
+ * |Y - Y_exact| <= 2^-7 |Y_exact| + 1e-4 sum_k |x_hat w_hat|.  The
+ * quantizers are bit-exact.
+ */
+#ifndef FGFP8_H
+#define FGFP8_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FGFP8_VERSION 1
+
+/* Scale storage ("Fine-grained FP8", "UE8M0 scale format"). */
+typedef enum {
+  FGFP8_SCALE_F32 = 0,   /* float32, 4 bytes per scale */
+  FGFP8_SCALE_UE8M0 = 1  /* float8_e8m0fnu: one byte e, value 2^(e-127); 0xFF = NaN */
+} fgfp8_scale_fmt;
+
+typedef enum {
+  FGFP8_OK = 0,
+  FGFP8_ERR_INVALID_ARG = 1, /* null pointer, bad enum, negative size */
+  FGFP8_ERR_SHAPE = 2,       /* K or N not a multiple of 128, ld too small, size too large */
+  FGFP8_ERR_ALIGN = 3,       /* a pointer or leading dimension breaks the 16-byte rule */
+  FGFP8_ERR_UNSUPPORTED = 4, /* a valid request this build does not implement */
+  FGFP8_ERR_CUDA = 5,        /* a CUDA runtime or driver call failed */
+  FGFP8_ERR_TIMEOUT = 6,     /* a kernel gave up on a barrier wait (device status) */
+  FGFP8_ERR_DEVICE = 7       /* a kernel rejected its device-side inputs (device status) */
+} fgfp8_status;
+
+/* FGFP8_VERSION of the loaded library. */
+int fgfp8_version(void);
+
+/* Message for the last error on the calling thread ("" if none).  The string
+ * is owned by the library.  It stays valid until the next call from the same
+ * thread. */
+const char* fgfp8_last_error_string(void);
+
+/*
+ * 128x128 block weight quantization ("Fine-grained FP8", introduction).
+ *   W   bf16 [N, K], row stride ldw elements (ldw >= K, ldw % 8 == 0,
+ *       16-byte aligned).
+ *   Wq  E4M3 codes [N, K], row stride K bytes, 16-byte aligned.
+ *   Ws  [N/128, K/128] row-major: float (fmt F32, 4-byte aligned) or UE8M0
+ *       bytes.  Ws[nb*(K/128) + kb] is the scale of rows nb*128.. and columns
+ *       kb*128..
+ * N % 128 == 0 and K % 128 == 0.  N == 0 is a no-op.  For a stack of E expert
+ * matrices, pass N = E * N_expert: blocks never straddle experts.
+ */
+fgfp8_status fgfp8_quant_weight(const void* W, int64_t N, int64_t K, int64_t ldw, uint8_t* Wq, void* Ws,
+                                int fmt, void* stream);
+
+/*
+ * Dynamic per-token activation quantization, groups of 128 along K
+ * ("Fine-grained FP8", introduction and "DeepGEMM fast path").
+ *   X   bf16 [M, K], row stride ldx elements (ldx >= K, ldx % 8 == 0,
+ *       16-byte aligned).
+ *   Xq  E4M3 codes [M, K], row stride K bytes, 16-byte aligned.
+ *   Xs  scales stored MN-major: the scale of token m, group g is
+ *       Xs[g*ld_s + m] (float for F32, byte for UE8M0).  ld_s >= M.  ld_s is
+ *       a multiple of 4 (F32) or 16 (UE8M0), and Xs is 16-byte aligned, so
+ *       each scale row is a valid TMA source.  Entries m >= M are not written.
+ * K % 128 == 0.  M == 0 is a no-op.
+ */
+fgfp8_status fgfp8_quant_act(const void* X, int64_t M, int64_t K, int64_t ldx, uint8_t* Xq, void* Xs,
+                             int64_t ld_s, int fmt, void* stream);
+
+/*
+ * Block-scaled FP8 GEMM, Y = X * W^T with both scales applied per 128-wide
+ * K block ("Fine-grained FP8", "DeepGEMM fast path": the FP8 linear layer).
+ *   Xq, Xs, ld_s  as written by fgfp8_quant_act (same fmt).
+ *   Wq, Ws        as written by fgfp8_quant_weight (same fmt).
+ *   Y             bf16 [M, N] row-major (row stride N), 16-byte aligned.
+ * K % 128 == 0, N % 128 == 0, M >= 0 arbitrary (M == 0 is a no-op).
+ * M, N, K < 2^31.
+ */
+fgfp8_status fgfp8_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
+                        void* Y, int64_t M, int64_t N, int64_t K, int fmt, void* stream);
+
+/*
+ * M-grouped GEMM for MoE experts ("Fine-grained FP8", "DeepGEMM fast path":
+ * the experts backend).  The rows of Xq are grouped per expert in
+ * contiguous segments: rows [group_offs[e], group_offs[e+1]) belong to
+ * expert e and are multiplied by Wq[e].
+ *   Xq, Xs, ld_s  as from fgfp8_quant_act over all M_total rows.
+ *   Wq            [E, N, K] E4M3 (E stacked fgfp8_quant_weight outputs).
+ *   Ws            [E, N/128, K/128].
+ *   Y             bf16 [M_total, N].
+ *   group_offs    DEVICE int32 [E+1]: group_offs[0] == 0,
+ *                 group_offs[E] == M_total, non-decreasing, every entry a
+ *                 multiple of 128.  Empty experts are allowed.
+ * Rows a caller padded with zeros produce zeros.  M_total % 128 == 0.  The
+ * offsets are checked on the device.  Inconsistent offsets leave the affected
+ * tiles unwritten, and fgfp8_check_device_status then reports
+ * FGFP8_ERR_DEVICE.  Both scale formats are accepted.
+ */
+fgfp8_status fgfp8_grouped_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq,
+                                const void* Ws, void* Y, const int32_t* group_offs, int32_t E,
+                                int64_t M_total, int64_t N, int64_t K, int fmt, void* stream);
+
+/*
+ * Synchronizes `stream`, then reads and clears the device status word that
+ * the kernels set when they give up.  It returns FGFP8_OK,
+ * FGFP8_ERR_TIMEOUT (a barrier wait ran past its one-second limit),
+ * FGFP8_ERR_DEVICE (inconsistent group offsets) or FGFP8_ERR_CUDA.
+ */
+fgfp8_status fgfp8_check_device_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FGFP8_H */

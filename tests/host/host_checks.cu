@@ -1,0 +1,77 @@
+// Host-only checks of two pieces of integer / floating-point arithmetic the
+// activation quantizer relies on (compiled with nvcc, run on the CPU):
+//  1. FastDiv (Granlund-Montgomery) equals integer division for every
+//     divisor 1..65536 on edge and random numerators;
+//  2. the FMA-based quotient q = fma(fma(-q0, s, a), r, q0), q0 = a*r,
+//     r = RN(1/s) equals the IEEE quotient RN(a/s) for EVERY pair the kernel
+//     meets: a = |x| for a bf16 x, s = RN(amax_c/448) for a bf16 amax >= |x|
+//     (amax_c = max(amax, 1e-4)), wherever the quotient can reach a nonzero
+//     E4M3 code.  E4M3 rounds every |v| <= 2^-10 to zero (2^-10 is halfway to
+//     the smallest subnormal 2^-9 and ties go to the even code 0), so below
+//     that only "both quotients <= 2^-10" is required; there the FMA residual
+//     of a subnormal |x| may be inexact.  Host fmaf/division/multiplication
+//     are IEEE round-to-nearest, like the device intrinsics the kernel uses.
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <random>
+
+#include "quant.cuh"
+
+static float bf16_bits_to_float(uint32_t h) {
+  uint32_t u = h << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+
+static uint32_t fbits(float f) {
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  return u;
+}
+
+int main() {
+  long bad = 0;
+  // ---- 1. FastDiv
+  std::mt19937_64 rng(1);
+  for (uint32_t d = 1; d <= 65536; ++d) {
+    fgfp8::FastDiv f(d);
+    const uint32_t edge[] = {0u, 1u, d - 1, d, d + 1, 2 * d - 1, 2 * d, 0x7FFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFEu};
+    for (uint32_t n : edge)
+      if (f.div(n) != n / d) ++bad;
+    for (int i = 0; i < 64; ++i) {
+      uint32_t n = static_cast<uint32_t>(rng());
+      if (f.div(n) != n / d) ++bad;
+    }
+  }
+  std::printf("fastdiv mismatches: %ld\n", bad);
+  if (bad) return 1;
+
+  // ---- 2. FMA-based quotient vs IEEE division, exhaustive over bf16 pairs
+  long pairs = 0, qbad = 0, below = 0;
+  const float zero_limit = 0x1p-10f;
+#pragma omp parallel for schedule(dynamic, 64) reduction(+ : pairs, qbad, below)
+  for (int64_t ab = 1; ab <= 0x7F7F; ++ab) {               // every positive finite bf16 amax
+    const float amax = bf16_bits_to_float(static_cast<uint32_t>(ab));
+    const float amax_c = amax < 1e-4f ? 1e-4f : amax;
+    const float s = amax_c / 448.0f;
+    const float r = 1.0f / s;
+    for (uint32_t h = 0; h <= static_cast<uint32_t>(ab); ++h) {   // every |x| <= amax
+      const float a = bf16_bits_to_float(h);
+      const float q0 = a * r;
+      const float e = std::fmaf(-q0, s, a);
+      const float q = std::fmaf(e, r, q0);
+      const float ref = a / s;
+      ++pairs;
+      if (q <= zero_limit && ref <= zero_limit) {
+        ++below;                                   // both encode to a zero code
+      } else if (fbits(q) != fbits(ref)) {
+        ++qbad;
+      }
+    }
+  }
+  std::printf("quotient pairs: %ld (of which %ld both <= 2^-10) mismatches: %ld\n", pairs, below, qbad);
+  return qbad ? 2 : 0;
+}

@@ -1,0 +1,112 @@
+"""The C ABI on the host (CPU only, no compute): the library loads, exports
+every symbol include/fgfp8.h declares, validates arguments before touching
+the GPU, and fails loudly (FGFP8_ERR_CUDA) instead of computing on the CPU
+when no usable GPU is present."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+import fine_grained_fp8_token_b200 as fg
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fgfp8.h")
+
+OK, INVALID, SHAPE, ALIGN, UNSUP, CUDA = 0, 1, 2, 3, 4, 5
+A = 1 << 20          # a fake, 16-byte aligned "device" address; never dereferenced on these paths
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:fgfp8_status|int|const char\*)\s+(fgfp8_\w+)\s*\(", text, re.M)))
+
+
+def test_library_builds_and_loads():
+    lib = fg.load()
+    assert lib.fgfp8_version() == 1
+
+
+def test_exports_every_declared_symbol():
+    names = declared_functions()
+    assert len(names) >= 7
+    assert set(names) == set(fg.SIGNATURES), "binding signatures and header disagree"
+    out = subprocess.run(["nm", "-D", "--defined-only", fg.library_path()], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r" T (fgfp8_\w+)$", out, re.M))
+    missing = set(names) - exported
+    assert not missing, f"declared but not exported: {missing}"
+
+
+def test_no_cpu_library_on_product_path():
+    """The product library links no oracle code and the package imports none."""
+    out = subprocess.run(["nm", "-D", fg.library_path()], capture_output=True, text=True, check=True).stdout
+    assert "orc_" not in out
+    src = open(os.path.join(ROOT, "fine_grained_fp8_token_b200", "__init__.py")).read()
+    assert "oracle" not in src.replace("# oracle", "")
+
+
+def st(code):
+    return code
+
+
+def test_quant_act_validation():
+    f = fg.fgfp8_quant_act
+    assert f(A, 4, 100, 100, A, A, 4, 0, None) == SHAPE                 # K % 128
+    assert f(A, 4, 256, 128, A, A, 4, 0, None) == SHAPE                 # ldx < K
+    assert f(A, 4, 256, 256, A, A, 2, 0, None) == SHAPE                 # ld_s < M
+    assert f(A, 4, 256, 256, A, A, 6, 0, None) == ALIGN                 # ld_s % 4 (fp32)
+    assert f(A, 4, 256, 256, A, A, 8, 1, None) == ALIGN                 # ld_s % 16 (ue8m0)
+    assert f(A, 4, 256, 256, A, A, 4, 2, None) == INVALID               # fmt
+    assert f(0, 4, 256, 256, A, A, 4, 0, None) == INVALID               # NULL X
+    assert f(A + 2, 4, 256, 256, A, A, 4, 0, None) == ALIGN             # X alignment
+    assert f(A, 4, 256, 260, A, A, 4, 0, None) == ALIGN                 # ldx % 8
+    assert f(A, 4, 256, 256, A + 8, A, 4, 0, None) == ALIGN             # Xq alignment
+    assert f(A, -1, 256, 256, A, A, 4, 0, None) == INVALID              # negative
+    assert f(A, 0, 256, 256, A, A, 4, 0, None) == OK                    # empty: no-op
+    assert "ld" in fg.fgfp8_last_error_string() or fg.fgfp8_last_error_string() == ""
+
+
+def test_quant_weight_validation():
+    f = fg.fgfp8_quant_weight
+    assert f(A, 100, 256, 256, A, A, 0, None) == SHAPE                  # N % 128
+    assert f(A, 128, 200, 256, A, A, 0, None) == SHAPE                  # K % 128
+    assert f(A, 128, 256, 128, A, A, 0, None) == SHAPE                  # ldw < K
+    assert f(A, 128, 256, 256, A, A + 2, 0, None) == ALIGN              # fp32 Ws alignment
+    assert f(A, 128, 256, 256, A, 0, 1, None) == INVALID                # NULL Ws
+    assert f(A, 0, 256, 256, A, A, 0, None) == OK
+
+
+def test_gemm_validation():
+    f = fg.fgfp8_gemm
+    assert f(A, A, 4, A, A, A, 4, 256, 100, 0, None) == SHAPE           # K
+    assert f(A, A, 4, A, A, A, 4, 200, 256, 0, None) == SHAPE           # N
+    assert f(A, A, 2, A, A, A, 4, 256, 256, 0, None) == SHAPE           # ld_s < M
+    assert f(A, A, 4, A, A, A + 8, 4, 256, 256, 0, None) == ALIGN       # Y
+    assert f(A, A + 4, 4, A, A, A, 4, 256, 256, 0, None) == ALIGN       # Xs 16-byte
+    assert f(A, A, 4, 0, A, A, 4, 256, 256, 0, None) == INVALID         # NULL Wq
+    assert f(A, A, 4, A, A, A, 4, 256, 256, 7, None) == INVALID         # fmt
+    assert f(A, A, 4, A, A, A, 1 << 31, 256, 256, 0, None) == SHAPE     # M too large (ld_s < M first)
+    assert f(A, A, 4, A, A, A, 0, 256, 256, 0, None) == OK              # empty
+
+
+def test_grouped_gemm_validation():
+    f = fg.fgfp8_grouped_gemm
+    assert f(A, A, 256, A, A, A, A, 0, 256, 256, 256, 1, None) == INVALID     # E
+    assert f(A, A, 256, A, A, A, A, 4, 200, 256, 256, 1, None) == SHAPE       # M_total % 128
+    assert f(A, A, 256, A, A, A, 0, 4, 256, 256, 256, 1, None) == INVALID     # NULL offsets
+    assert f(A, A, 256, A, A, A, A + 2, 4, 256, 256, 256, 1, None) == ALIGN   # offsets alignment
+    assert f(A, A, 256, A, A, A, A, 4, 0, 256, 256, 1, None) == OK            # empty
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the behaviour without a GPU")
+def test_valid_call_without_gpu_fails_loudly():
+    """No CPU fallback: a well-formed request on a machine without an
+    sm_100a GPU returns FGFP8_ERR_CUDA and launches nothing."""
+    assert fg.fgfp8_quant_act(A, 4, 256, 256, A, A, 4, 0, None) == CUDA
+    assert "cuda" in fg.fgfp8_last_error_string().lower()
+    assert fg.fgfp8_gemm(A, A, 4, A, A, A, 4, 256, 256, 0, None) == CUDA
+    with pytest.raises(fg.FGFP8Error):
+        fg._check(fg.fgfp8_quant_weight(A, 128, 256, 256, A, A, 0, None), "quant_weight")

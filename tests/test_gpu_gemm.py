@@ -1,0 +1,197 @@
+"""GPU parity of the block-scaled GEMM and the M-grouped GEMM against the
+oracle: every output within |gpu - ref| <= 2^-7 |ref| + 1e-4 sum_k |x_hat w_hat|.
+
+The GPU path and the oracle each quantize the same seeded bf16 inputs on
+their own (their codes are bit-identical, checked in test_gpu_quant.py), then
+multiply; no oracle input comes from the GPU."""
+import numpy as np
+import pytest
+import torch
+
+import fine_grained_fp8_token_b200 as fg
+import oracle
+import workloads
+from parity import F32, UE8M0, assert_gemm_close, bits16, require_gpu, to_np, y_to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dev():
+    d = require_gpu()
+    fg.load()
+    return d
+
+
+def gpu_linear(X_dev, W_dev, fmt):
+    Xq, Xs = fg.quant_act(X_dev, fmt)
+    Wq, Ws = fg.quant_weight(W_dev, fmt)
+    Y = fg.gemm(Xq, Xs, Wq, Ws, fmt)
+    fg.check_device_status()
+    return Y
+
+
+def oracle_linear(X_bits, W_bits, fmt, rows=None):
+    Wq, Ws = oracle.quant_weight(W_bits, fmt)
+    if rows is not None:
+        X_bits = X_bits[rows]
+    Xq, Xs = oracle.quant_act(X_bits, fmt)
+    return oracle.gemm(Xq, Xs, Wq, Ws, fmt)
+
+
+SMALL = [(128, 256, 512), (1, 128, 128), (7, 256, 384), (129, 384, 1024), (300, 640, 2048),
+         (513, 512, 4096), (64, 1280, 7168), (256, 2304, 256), (17, 128, 14336)]
+
+
+@pytest.mark.parametrize("fmt", [F32, UE8M0])
+@pytest.mark.parametrize("M,N,K", SMALL)
+def test_gemm_small(dev, fmt, M, N, K):
+    cfg = workloads.scaled_linear(workloads.TINY, M=M, N=N, K=K, seed=M + 3 * N + 7 * K)
+    X, W = workloads.linear_inputs(cfg)
+    Y = gpu_linear(X.to(dev), W.to(dev), fmt)
+    Y_ref, S = oracle_linear(bits16(X), bits16(W), fmt)
+    assert_gemm_close(y_to_f64(Y), Y_ref, S, f"gemm {M}x{N}x{K}")
+
+
+def test_gemm_tiny_config_exact_shape(dev):
+    """The tiny parity configuration, every output element."""
+    cfg = workloads.TINY
+    X, W = workloads.linear_inputs(cfg)
+    Y = gpu_linear(X.to(dev), W.to(dev), cfg.fmt)
+    Y_ref, S = oracle_linear(bits16(X), bits16(W), cfg.fmt)
+    assert_gemm_close(y_to_f64(Y), Y_ref, S, cfg.name)
+
+
+def test_gemm_repeatable(dev):
+    cfg = workloads.scaled_linear(workloads.TINY, M=300, N=512, K=1024)
+    X, W = workloads.linear_inputs(cfg)
+    Y1 = gpu_linear(X.to(dev), W.to(dev), F32)
+    Y2 = gpu_linear(X.to(dev), W.to(dev), F32)
+    assert torch.equal(Y1, Y2)
+
+
+def test_gemm_zero_and_unit_codes(dev):
+    """All codes 1.0 with unit scales gives K exactly; zero codes give 0."""
+    M, N, K = 130, 256, 1024
+    Xq = torch.full((M, K), 0x38, dtype=torch.uint8, device=dev)
+    Wq = torch.full((N, K), 0x38, dtype=torch.uint8, device=dev)
+    Xs = torch.ones((K // 128, fg.scale_rows(M, F32)), dtype=torch.float32, device=dev)
+    Ws = torch.ones((N // 128, K // 128), dtype=torch.float32, device=dev)
+    Y = fg.gemm(Xq, Xs, Wq, Ws, F32)
+    assert (Y.float() == K).all()
+    Y = fg.gemm(torch.zeros_like(Xq), Xs, Wq, Ws, F32)
+    assert (Y.float() == 0).all()
+
+
+def sample_rows(M, n_random=48, seed=0):
+    rng = np.random.default_rng(seed)
+    tiles = np.arange(0, M, 128)
+    rows = np.concatenate([tiles, np.minimum(tiles + 127, M - 1), rng.integers(0, M, n_random)])
+    return np.unique(rows)
+
+
+@pytest.mark.parametrize("cfg", [workloads.LLAMA_ATTN, workloads.LLAMA_GATE_UP, workloads.LLAMA_DOWN],
+                         ids=lambda c: c.name)
+def test_gemm_full_size_sampled_rows(dev, cfg):
+    X = workloads.activations((cfg.M, cfg.K), cfg.x_kind, cfg.seed, device=dev)
+    W = workloads.weights((cfg.N, cfg.K), cfg.seed + 1, device=dev)
+    Y = gpu_linear(X, W, cfg.fmt)
+    rows = sample_rows(cfg.M, n_random=16 if cfg.N > 8192 else 48)
+    if cfg.N > 8192:
+        rows = rows[::2]
+    Y_ref, S = oracle_linear(bits16(X), bits16(W), cfg.fmt, rows=rows)
+    assert_gemm_close(y_to_f64(Y[torch.as_tensor(rows, device=dev)]), Y_ref, S, cfg.name)
+
+
+@pytest.mark.parametrize("m", [1, 8, 32, 64])
+def test_gemm_decode_ue8m0(dev, m):
+    cfg = workloads.DS_DECODE[m]
+    X = workloads.activations((cfg.M, cfg.K), cfg.x_kind, cfg.seed, device=dev)
+    W = workloads.weights((cfg.N, cfg.K), cfg.seed + 1, device=dev)
+    Y = gpu_linear(X, W, cfg.fmt)
+    rows = np.arange(cfg.M) if cfg.M <= 8 else np.unique(np.r_[0, cfg.M - 1, np.arange(1, cfg.M, 5)])
+    Y_ref, S = oracle_linear(bits16(X), bits16(W), cfg.fmt, rows=rows)
+    assert_gemm_close(y_to_f64(Y[torch.as_tensor(rows, device=dev)]), Y_ref, S, cfg.name)
+
+
+# ---------------------------------------------------------------- grouped
+def build_moe(cfg, dev):
+    r = workloads.moe_routing(cfg)
+    X = workloads.moe_grouped_rows(workloads.moe_tokens(cfg, device=dev), r)
+    Wq = torch.empty((cfg.E, cfg.N, cfg.K), dtype=torch.uint8, device=dev)
+    Ws = torch.empty((cfg.E, cfg.N // 128, cfg.K // 128), dtype=torch.float32 if cfg.fmt == F32 else torch.uint8,
+                     device=dev)
+    for e in range(cfg.E):
+        fg.quant_weight(workloads.moe_expert_weight(cfg, e, device=dev), cfg.fmt, Wq=Wq[e], Ws=Ws[e])
+    Xq, Xs = fg.quant_act(X, cfg.fmt)
+    offs = torch.as_tensor(r.group_offs, device=dev)
+    Y = fg.grouped_gemm(Xq, Xs, Wq, Ws, offs, cfg.fmt)
+    fg.check_device_status()
+    return r, X, Y
+
+
+def oracle_moe_rows(cfg, r, X, rows, dev):
+    Y_ref = np.empty((len(rows), cfg.N))
+    S = np.empty((len(rows), cfg.N))
+    expert_of = np.searchsorted(r.group_offs, rows, side="right") - 1
+    X_rows = bits16(X[torch.as_tensor(rows, device=dev)])
+    for e in np.unique(expert_of):
+        sel = np.where(expert_of == e)[0]
+        W = workloads.moe_expert_weight(cfg, int(e), device=dev)
+        y, s = oracle_linear(X_rows, bits16(W), cfg.fmt, rows=sel)
+        Y_ref[sel], S[sel] = y, s
+    return Y_ref, S
+
+
+@pytest.mark.parametrize("fmt", [UE8M0, F32])
+def test_grouped_gemm_small(dev, fmt):
+    cfg = workloads.scaled_moe(workloads.MOE, E=9, N=256, K=512, tokens=300, topk=3, fmt=fmt)
+    r, X, Y = build_moe(cfg, dev)
+    valid = np.where(r.row_token >= 0)[0]
+    Y_ref, S = oracle_moe_rows(cfg, r, X, valid, dev)
+    assert_gemm_close(y_to_f64(Y[torch.as_tensor(valid, device=dev)]), Y_ref, S, "grouped small")
+    pad = torch.as_tensor(np.where(r.row_token < 0)[0], device=dev)
+    assert (Y[pad].float() == 0).all()
+
+
+def test_grouped_gemm_empty_experts(dev):
+    """Experts with no rows (zero-length segments) are skipped."""
+    cfg = workloads.scaled_moe(workloads.MOE, E=40, N=128, K=256, tokens=20, topk=1, zipf=3.0)
+    r, X, Y = build_moe(cfg, dev)
+    assert (r.counts == 0).any()
+    valid = np.where(r.row_token >= 0)[0]
+    Y_ref, S = oracle_moe_rows(cfg, r, X, valid, dev)
+    assert_gemm_close(y_to_f64(Y[torch.as_tensor(valid, device=dev)]), Y_ref, S, "grouped empty experts")
+
+
+def test_grouped_gemm_full_moe_sampled_rows(dev):
+    cfg = workloads.MOE
+    r, X, Y = build_moe(cfg, dev)
+    starts = r.group_offs[:-1]
+    big = np.argsort(-r.counts)[:3]
+    pick = np.unique(np.r_[big, [cfg.E // 2, cfg.E - 1, 100]])
+    rows = []
+    for e in pick:
+        lo, n = int(starts[e]), int(r.counts[e])
+        rows += [lo, lo + n - 1, lo + n // 2]
+    rows = np.unique(np.array(rows))
+    Y_ref, S = oracle_moe_rows(cfg, r, X, rows, dev)
+    assert_gemm_close(y_to_f64(Y[torch.as_tensor(rows, device=dev)]), Y_ref, S, cfg.name)
+
+
+def test_grouped_gemm_bad_offsets_reported(dev):
+    """Offsets that do not cover the rows are rejected on the device: the
+    affected tiles stay unwritten and the status reads FGFP8_ERR_DEVICE."""
+    E, N, K, M = 2, 128, 256, 256
+    Xq = torch.zeros((M, K), dtype=torch.uint8, device=dev)
+    Xs = torch.ones((K // 128, M), dtype=torch.uint8, device=dev) * 127
+    Wq = torch.zeros((E, N, K), dtype=torch.uint8, device=dev)
+    Ws = torch.full((E, 1, K // 128), 127, dtype=torch.uint8, device=dev)
+    offs = torch.tensor([0, 128, 128], dtype=torch.int32, device=dev)     # row block 1 uncovered
+    Y = torch.full((M, N), 7.0, dtype=torch.bfloat16, device=dev)
+    fg.grouped_gemm(Xq, Xs, Wq, Ws, offs, UE8M0, Y=Y)
+    with pytest.raises(fg.FGFP8Error) as ei:
+        fg.check_device_status()
+    assert ei.value.status == 7
+    assert (Y[:128].float() == 0).all() and (Y[128:].float() == 7).all()
+    fg.check_device_status()       # the status word was cleared
