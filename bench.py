@@ -12,7 +12,8 @@ Default workload: the Llama-3-8B attention projection in prefill,
 X [4096, 4096] x W [4096, 4096], fp32 block scales.  Other workloads can be
 chosen with --workload (see workloads/).
 
-Timing: W warm-up steps, then K timed steps.  L2 is flushed (a 256 MB write)
+Timing: W warm-up steps, then K timed steps.  L2 is flushed (a 256 MB write followed
+by a 256 MB read, so no dirty line is written back inside the next step)
 before every step, outside the timed events.  Each kernel is bracketed by
 CUDA events on the launching stream.  For N > 1 (torchrun) every rank runs
 its own replica of the workload with no collective on the data path, and
@@ -67,69 +68,76 @@ def measured_peaks():
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples of the GPU's clocks and throttle reasons during the
-    timed region."""
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    """SM clock and throttle reasons of this GPU, sampled every 10 ms through
+    NVML (read-only queries) while the timed region runs."""
 
     def __init__(self, device_index: int):
-        self.proc = None
-        self.path = None
+        self.ok = False
+        self.samples = []
         try:
-            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
-            ids = subprocess.run(["nvidia-smi", "--query-gpu=index,uuid", "--format=csv,noheader"],
-                                 capture_output=True, text=True, timeout=20).stdout
-            self.index = None
-            for line in ids.strip().splitlines():
-                idx, u = [x.strip() for x in line.split(",")]
-                if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
-                    self.index = idx
-            if self.index is None:
-                self.index = str(device_index)
+            import threading
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid).replace("GPU-", "")
+            handle = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(h)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == uuid:
+                    handle = h
+            if handle is None:
+                return
+            self.nv, self.h, self.threading = pynvml, handle, threading
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+            self.ok = True
         except Exception:
-            self.index = None
+            self.ok = False
+
+    def _loop(self):
+        nv = self.nv
+        while not self.stop_flag.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, reasons))
+            except Exception:
+                pass
+            self.stop_flag.wait(0.01)
 
     def start(self):
-        if self.index is None:
+        if not self.ok:
             return
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
-        try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.index, f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+        self.stop_flag = self.threading.Event()
+        self.thread = self.threading.Thread(target=self._loop, daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if self.proc is None:
+        if not self.ok:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=10)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        rows = []
-        for line in open(self.path).read().strip().splitlines():
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                rows.append((float(parts[0]), float(parts[1]), parts[3:]))
-            except ValueError:
-                continue
-        os.unlink(self.path)
-        if not rows:
+        self.stop_flag.set()
+        self.thread.join(timeout=5)
+        if not self.samples:
             return None
-        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = set()
-        for _, _, flags in rows:
-            for n, v in zip(names[1:], flags[1:]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
-                "samples": len(rows), "reasons": sorted(reasons)}
+        nv = self.nv
+        names = {"hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+                 "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+                 "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+                 "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4)}
+        seen = set()
+        for _, r in self.samples:
+            for n, bit in names.items():
+                if r & bit:
+                    seen.add(n)
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "samples": len(self.samples), "reasons": sorted(seen)}
+
+
+def flush_l2(buf_w, buf_r):
+    """Evict L2: write a buffer larger than L2, then read another one so the
+    lines left behind are clean (no write-back lands in the next kernel)."""
+    buf_w.fill_(1)
+    buf_r.sum(dtype=torch.int32)
 
 
 # ---------------------------------------------------------------- workloads on the GPU
@@ -256,7 +264,8 @@ def make_layer(name, dev):
 def run_gpu(args, rank, world, dev):
     layer = make_layer(args.workload, dev)
     stream = torch.cuda.current_stream(dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
     launches_per_step = 2
 
     def step():
@@ -264,7 +273,7 @@ def run_gpu(args, rank, world, dev):
         layer.gemm()
 
     for _ in range(args.warmup):
-        flush.fill_(1)
+        flush_l2(flush_w, flush_r)
         step()
     layer.fg.check_device_status()
 
@@ -276,7 +285,7 @@ def run_gpu(args, rank, world, dev):
     torch.cuda.synchronize(dev)
     sampler.start()
     for i in range(n):
-        flush.fill_(1)
+        flush_l2(flush_w, flush_r)
         ev[i][0].record(stream)
         layer.quant_act()
         ev[i][1].record(stream)
@@ -295,7 +304,7 @@ def run_gpu(args, rank, world, dev):
     # weight quantization (offline step, reported, not part of the step)
     wq_ms = []
     for _ in range(max(3, min(n, 10))):
-        flush.fill_(1)
+        flush_l2(flush_w, flush_r)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         layer.quant_weight()
@@ -313,7 +322,7 @@ def run_gpu(args, rank, world, dev):
     e2e_ms = []
     e2e_steps = max(3, min(n, 10))
     for i in range(e2e_steps + 2):
-        flush.fill_(1)
+        flush_l2(flush_w, flush_r)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         X_stage.copy_(X_host, non_blocking=True)
@@ -436,7 +445,7 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="fgfp8", choices=["fgfp8", "reference"])
     ap.add_argument("--workload", default="llama_attn",
@@ -486,7 +495,7 @@ def main():
         "impl": "fgfp8", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": n,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "e4m3xe4m3->f32", "data": "synthetic (seeded, see workloads/)",
-        "config": {**layer.describe(), "l2": "flushed (256 MB write) before every timed step",
+        "config": {**layer.describe(), "l2": "flushed before every timed step (256 MB write, then 256 MB read)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": roofline,
         "kernels": {

@@ -156,6 +156,34 @@ fgfp8_status launch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const 
   return check_launch("gemm launch");
 }
 
+// Few-token (M <= 64) launch: one CTA per 128 output columns, operands swapped.
+template <int BNT, int FMT>
+fgfp8_status launch_decode(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
+                           void* Y, int64_t M, int64_t N, int64_t K, cudaStream_t stream, int dev) {
+  using C = fgfp8::DecodeCfg<BNT>;
+  CUtensorMap mX, mW;
+  fgfp8_status st = make_map_u8_sw128(&mX, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
+                                      static_cast<uint64_t>(K), BNT);
+  if (st != FGFP8_OK) return st;
+  st = make_map_u8_sw128(&mW, Wq, static_cast<uint64_t>(N), static_cast<uint64_t>(K), static_cast<uint64_t>(K), 128);
+  if (st != FGFP8_OK) return st;
+  auto kernel = fgfp8::gemm_decode_kernel<BNT, FMT>;
+  st = set_smem(reinterpret_cast<const void*>(kernel), C::kSmemBytes, dev);
+  if (st != FGFP8_OK) return st;
+  kernel<<<static_cast<unsigned>(N / 128), C::kThreads, C::kSmemBytes, stream>>>(
+      mX, mW, Xs, static_cast<uint32_t>(ld_s), Ws, reinterpret_cast<__nv_bfloat16*>(Y), static_cast<int>(M),
+      static_cast<int>(N), static_cast<int>(K));
+  return check_launch("decode gemm launch");
+}
+
+template <int FMT>
+fgfp8_status dispatch_decode(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
+                             void* Y, int64_t M, int64_t N, int64_t K, cudaStream_t s, int dev) {
+  if (M <= 16) return launch_decode<16, FMT>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev);
+  if (M <= 32) return launch_decode<32, FMT>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev);
+  return launch_decode<64, FMT>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev);
+}
+
 template <bool kGrouped>
 fgfp8_status dispatch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws, void* Y,
                            int64_t M, int64_t N, int64_t K, int fmt, const int32_t* offs, int E, int64_t b_rows,
@@ -279,8 +307,12 @@ fgfp8_status fgfp8_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const u
   DeviceInfo info;
   st = current_device(&dev, &info);
   if (st != FGFP8_OK) return st;
-  return dispatch_gemm<false>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, fmt, nullptr, 1, N,
-                              reinterpret_cast<cudaStream_t>(stream), dev);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (M <= 64) {
+    return fmt == FGFP8_SCALE_F32 ? dispatch_decode<0>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev)
+                                  : dispatch_decode<1>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev);
+  }
+  return dispatch_gemm<false>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, fmt, nullptr, 1, N, s, dev);
 }
 
 fgfp8_status fgfp8_grouped_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,

@@ -83,6 +83,71 @@ __device__ __forceinline__ int find_expert(const int32_t* __restrict__ offs, int
   return -1;
 }
 
+// ---------------------------------------------------------------------------
+// Pipeline roles shared by the GEMM kernels.
+// ---------------------------------------------------------------------------
+
+// TMA producer (one thread): per K block, a kABytes tile of operand A (rows
+// a_row.., box from tmA) and a kBBytes tile of operand B into ring slot
+// kb % kStages; waits for the slot to be released by the MMA first.  Before
+// returning it waits for every copy it issued to land.
+template <int kStages, uint32_t kABytes, uint32_t kBBytes>
+__device__ __forceinline__ void produce_tiles(const CUtensorMap* tmA, int a_row, const CUtensorMap* tmB, int b_row,
+                                              int KB, uint8_t* sA, uint8_t* sB, uint64_t* full, uint64_t* empty) {
+  int issued = 0;
+  for (int kb = 0; kb < KB; ++kb) {
+    const int s = kb % kStages;
+    const uint32_t use = kb / kStages;
+    if (kb >= kStages && !mbar_wait(&empty[s], (use & 1u) ^ 1u)) {
+      record_status(kDevTimeoutProducer);
+      break;
+    }
+    mbar_arrive_expect_tx(&full[s], kABytes + kBBytes);
+    tma_load_2d(sA + s * kABytes, tmA, &full[s], kb * 128, a_row);
+    tma_load_2d(sB + s * kBBytes, tmB, &full[s], kb * 128, b_row);
+    issued = kb + 1;
+  }
+  for (int kb = (issued > kStages ? issued - kStages : 0); kb < issued; ++kb) {
+    if (!mbar_wait(&full[kb % kStages], (kb / kStages) & 1u)) record_status(kDevTimeoutProducer);
+  }
+}
+
+// MMA issuer (one thread): per K block, four K=32 tcgen05.mma (M=128, N=kN)
+// into TMEM partial buffer kb & 1 (columns [b*kN, b*kN + kN)), overwriting it
+// on the first step; then frees the smem slot and publishes the buffer.  The
+// buffer is reused only after the promotion warps released it.  A final
+// commit makes every MMA complete before the caller may free TMEM.
+template <int kStages, uint32_t kABytes, uint32_t kBBytes, int kN>
+__device__ __forceinline__ void issue_mmas(uint32_t a_base, uint32_t b_base, int KB, uint32_t tmem_base,
+                                           uint64_t* full, uint64_t* empty, uint64_t* tfull, uint64_t* tempty,
+                                           uint64_t* mma_done) {
+  constexpr uint32_t idesc = idesc_e4m3_f32(128, kN);
+  for (int kb = 0; kb < KB; ++kb) {
+    const int s = kb % kStages;
+    const int b = kb & 1;
+    if (!mbar_wait(&full[s], (kb / kStages) & 1u)) {
+      record_status(kDevTimeoutMma);
+      break;
+    }
+    if (kb >= 2 && !mbar_wait(&tempty[b], ((kb >> 1) & 1u) ^ 1u)) {
+      record_status(kDevTimeoutMma);
+      break;
+    }
+    tc_fence_after();
+    const uint32_t d = tmem_base + static_cast<uint32_t>(b * kN);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const uint64_t ad = smem_desc_k_sw128(a_base + s * kABytes + kk * 32);
+      const uint64_t bd = smem_desc_k_sw128(b_base + s * kBBytes + kk * 32);
+      mma_f8f6f4(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
+    }
+    mma_commit(&empty[s]);
+    mma_commit(&tfull[b]);
+  }
+  mma_commit(mma_done);
+  if (!mbar_wait(mma_done, 0)) record_status(kDevTimeoutMma);
+}
+
 template <int BN, int FMT, bool kGrouped>
 __global__ void __launch_bounds__(GemmCfg<BN>::kThreads, 1)
     gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -156,57 +221,13 @@ __global__ void __launch_bounds__(GemmCfg<BN>::kThreads, 1)
 
   if (warp == 0) {
     // ================= TMA producer
-    if (lane == 0) {
-      const int b_row0 = expert * N + n0;
-      int issued = 0;
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % C::kStages;
-        const uint32_t use = kb / C::kStages;
-        if (kb >= C::kStages && !mbar_wait(&empty[s], (use & 1u) ^ 1u)) {
-          record_status(kDevTimeoutProducer);
-          break;
-        }
-        mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-        tma_load_2d(sA + s * C::kABytes, &tmA, &full[s], kb * C::kBK, m0);
-        tma_load_2d(sB + s * C::kBBytes, &tmB, &full[s], kb * C::kBK, b_row0);
-        issued = kb + 1;
-      }
-      // every copy issued must have landed before the CTA may exit
-      for (int kb = (issued > C::kStages ? issued - C::kStages : 0); kb < issued; ++kb) {
-        if (!mbar_wait(&full[kb % C::kStages], (kb / C::kStages) & 1u)) record_status(kDevTimeoutProducer);
-      }
-    }
+    if (lane == 0)
+      produce_tiles<C::kStages, C::kABytes, C::kBBytes>(&tmA, m0, &tmB, expert * N + n0, KB, sA, sB, full, empty);
   } else if (warp == 1) {
     // ================= MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(128, BN);
-      const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % C::kStages;
-        const int b = kb & 1;
-        if (!mbar_wait(&full[s], (kb / C::kStages) & 1u)) {
-          record_status(kDevTimeoutMma);
-          break;
-        }
-        if (kb >= 2 && !mbar_wait(&tempty[b], ((kb >> 1) & 1u) ^ 1u)) {
-          record_status(kDevTimeoutMma);
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d = tmem_base + static_cast<uint32_t>(b * BN);
-#pragma unroll
-        for (int kk = 0; kk < C::kBK / 32; ++kk) {
-          const uint64_t ad = smem_desc_k_sw128(a_base + s * C::kABytes + kk * 32);
-          const uint64_t bd = smem_desc_k_sw128(b_base + s * C::kBBytes + kk * 32);
-          mma_f8f6f4(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&empty[s]);
-        mma_commit(&tfull[b]);
-      }
-      // all MMAs of this thread complete before TMEM may be freed
-      mma_commit(mma_done);
-      if (!mbar_wait(mma_done, 0)) record_status(kDevTimeoutMma);
-    }
+    if (lane == 0)
+      issue_mmas<C::kStages, C::kABytes, C::kBBytes, BN>(smem_u32(sA), smem_u32(sB), KB, tmem_base, full, empty,
+                                                         tfull, tempty, mma_done);
   } else {
     // ================= promotion / epilogue
     const int ew = warp - 2;
@@ -274,6 +295,164 @@ __global__ void __launch_bounds__(GemmCfg<BN>::kThreads, 1)
   }
 
   // ---- teardown
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+
+// ---------------------------------------------------------------------------
+// Few-token variant (M <= 64, decode): operands swapped so the weight supplies
+// the MMA's 128 rows and the tokens its N dimension (BNT = M rounded up to
+// 16/32/64).  One CTA streams one 128-row weight slab through a deep TMA ring
+// (the layer is bound by reading Wq from HBM).  TMEM holds D^T: lane = output
+// column n, column = token m.  Each promotion thread owns one n and BNT
+// accumulators; the token scales sa[m, kb] are fetched once per warp
+// (one per lane) and broadcast with shuffles.
+// ---------------------------------------------------------------------------
+template <int BNT>
+struct DecodeCfg {
+  static constexpr uint32_t kABytes = 128 * 128;             // weight tile
+  static constexpr uint32_t kBBytes = BNT * 128;             // token tile
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = (200 * 1024) / kStageBytes > 12 ? 12 : (200 * 1024) / kStageBytes;
+  static constexpr int kThreads = 6 * 32;                    // producer, MMA, 4 promotion warps
+  static constexpr uint32_t kTmemCols = (2 * BNT < 32) ? 32 : 2 * BNT;
+  static constexpr size_t kSmemBytes = 1024 + kStages * static_cast<size_t>(kStageBytes) + 256;
+};
+
+template <int FMT>
+__device__ __forceinline__ uint32_t load_scale_raw(const void* __restrict__ p, uint64_t i) {
+  if (FMT == 0) return __float_as_uint(__ldg(reinterpret_cast<const float*>(p) + i));
+  return __ldg(reinterpret_cast<const uint8_t*>(p) + i);
+}
+
+// sa * sw from raw scale words (fp32 bits or UE8M0 bytes).
+template <int FMT>
+__device__ __forceinline__ float combine_raw(uint32_t a, uint32_t w) {
+  if (FMT == 0) return __uint_as_float(a) * __uint_as_float(w);
+  const int e = static_cast<int>(a) + static_cast<int>(w) - 127;
+  if (e >= 1 && e <= 254) return __int_as_float(e << 23);
+  return ldexpf(1.0f, static_cast<int>(a) + static_cast<int>(w) - 254);
+}
+
+template <int BNT, int FMT>
+__global__ void __launch_bounds__(DecodeCfg<BNT>::kThreads, 1)
+    gemm_decode_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                       const void* __restrict__ Xs, uint32_t ld_s, const void* __restrict__ Ws,
+                       __nv_bfloat16* __restrict__ Y, int M, int N, int K) {
+  using C = DecodeCfg<BNT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sW = smem;
+  uint8_t* sX = smem + C::kStages * C::kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sX + C::kStages * C::kBBytes);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* mma_done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int KB = K / 128;
+  const int n0 = blockIdx.x * 128;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    mbar_init(mma_done, 1);
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0)
+      produce_tiles<C::kStages, C::kABytes, C::kBBytes>(&tmW, n0, &tmX, 0, KB, sW, sX, full, empty);
+  } else if (warp == 1) {
+    if (lane == 0)
+      issue_mmas<C::kStages, C::kABytes, C::kBBytes, BNT>(smem_u32(sW), smem_u32(sX), KB, tmem_base, full, empty,
+                                                          tfull, tempty, mma_done);
+  } else {
+    const int quad = warp & 3;
+    const int n = n0 + quad * 32 + lane;
+    const uint64_t ws_row = static_cast<uint64_t>(n0 / 128) * KB;
+    const uint32_t taddr0 = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+    constexpr int kT = (BNT + 31) / 32;              // scale words per lane
+
+    float acc[BNT];
+#pragma unroll
+    for (int j = 0; j < BNT; ++j) acc[j] = 0.0f;
+
+    // raw scales of block kb: lane l holds the token scales l, l+32 (if < M)
+    auto load_scales = [&](int kb, uint32_t (&sa)[kT], uint32_t& sw) {
+#pragma unroll
+      for (int t = 0; t < kT; ++t) {
+        const int m = t * 32 + lane;
+        sa[t] = m < M ? load_scale_raw<FMT>(Xs, static_cast<uint64_t>(kb) * ld_s + m) : 0u;
+      }
+      sw = load_scale_raw<FMT>(Ws, ws_row + kb);
+    };
+
+    bool ok = true;
+    uint32_t sa_next[kT], sw_next;
+    load_scales(0, sa_next, sw_next);
+    for (int kb = 0; kb < KB; ++kb) {
+      const int b = kb & 1;
+      uint32_t sa[kT];
+#pragma unroll
+      for (int t = 0; t < kT; ++t) sa[t] = sa_next[t];
+      const uint32_t sw = sw_next;
+      if (kb + 1 < KB) load_scales(kb + 1, sa_next, sw_next);
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[b], (kb >> 1) & 1u))) {
+        if (lane == 0) record_status(kDevTimeoutEpilogue);
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = taddr0 + static_cast<uint32_t>(b * BNT);
+#pragma unroll
+      for (int c = 0; c < BNT / 16; ++c) {
+        uint32_t p[16];
+        tmem_ld_32x32b_x16(taddr + c * 16, p);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int m = c * 16 + j;
+          const uint32_t a = __shfl_sync(0xFFFFFFFFu, sa[m / 32], m % 32);
+          const float sc = (m < M) ? combine_raw<FMT>(a, sw) : 0.0f;
+          acc[m] = __fmaf_rn(__uint_as_float(p[j]), sc, acc[m]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[b]);
+    }
+    if (ok && n < N) {
+#pragma unroll
+      for (int m = 0; m < BNT; ++m)
+        if (m < M) Y[static_cast<uint64_t>(m) * N + n] = __float2bfloat16_rn(acc[m]);
+    }
+  }
+
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
