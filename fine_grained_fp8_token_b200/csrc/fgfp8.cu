@@ -132,12 +132,12 @@ fgfp8_status check_act_scales(const void* Xs, int64_t ld_s, int64_t M, int fmt) 
   return FGFP8_OK;
 }
 
-// Launch one GEMM instantiation.
-template <int BN, int FMT, bool kGrouped>
+// Launch one GEMM instantiation as a persistent grid (one CTA per SM at most).
+template <int BN, int CW, int FMT, bool kGrouped>
 fgfp8_status launch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
                          void* Y, int64_t M, int64_t N, int64_t K, const int32_t* offs, int E, int64_t b_rows,
-                         cudaStream_t stream, int dev) {
-  using C = fgfp8::GemmCfg<BN>;
+                         cudaStream_t stream, int dev, int sm_count) {
+  using C = fgfp8::GemmCfg<BN, CW>;
   CUtensorMap mA, mB;
   fgfp8_status st = make_map_u8_sw128(&mA, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
                                       static_cast<uint64_t>(K), 128);
@@ -145,15 +145,42 @@ fgfp8_status launch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const 
   st = make_map_u8_sw128(&mB, Wq, static_cast<uint64_t>(b_rows), static_cast<uint64_t>(K), static_cast<uint64_t>(K),
                          BN);
   if (st != FGFP8_OK) return st;
-  auto kernel = fgfp8::gemm_blockscaled_kernel<BN, FMT, kGrouped>;
+  auto kernel = fgfp8::gemm_blockscaled_kernel<BN, CW, FMT, kGrouped>;
   st = set_smem(reinterpret_cast<const void*>(kernel), C::kSmemBytes, dev);
   if (st != FGFP8_OK) return st;
   const int64_t tiles = ((M + C::kBM - 1) / C::kBM) * (N / BN);
   if (tiles == 0) return ok();
-  kernel<<<static_cast<unsigned>(tiles), C::kThreads, C::kSmemBytes, stream>>>(
+  const int64_t grid = tiles < sm_count ? tiles : sm_count;
+  kernel<<<static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, stream>>>(
       mA, mB, Xs, static_cast<uint32_t>(ld_s), Ws, reinterpret_cast<__nv_bfloat16*>(Y), static_cast<int>(M),
-      static_cast<int>(N), static_cast<int>(K), offs, E);
+      static_cast<int>(N), static_cast<int>(K), offs, E, static_cast<int>(tiles));
   return check_launch("gemm launch");
+}
+
+// Fraction of the last wave's CTA slots that hold work, for `tiles` tiles
+// spread over `sms` persistent CTAs.
+double wave_efficiency(int64_t tiles, int sms) {
+  const int64_t waves = (tiles + sms - 1) / sms;
+  return waves ? static_cast<double>(tiles) / static_cast<double>(waves * sms) : 1.0;
+}
+
+template <bool kGrouped>
+fgfp8_status dispatch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws, void* Y,
+                           int64_t M, int64_t N, int64_t K, int fmt, const int32_t* offs, int E, int64_t b_rows,
+                           cudaStream_t s, int dev, int sms) {
+  // 128x256 tiles halve the B traffic per MMA FLOP; 128x128 tiles when N is
+  // not a multiple of 256 or when they fill the last wave noticeably better.
+  const int64_t mt = (M + 127) / 128;
+  bool wide = (N % 256 == 0) && wave_efficiency(mt * (N / 256), sms) + 0.03 >= wave_efficiency(mt * (N / 128), sms);
+#if defined(FGFP8_FORCE_BN)
+  wide = (FGFP8_FORCE_BN == 256) && (N % 256 == 0);
+#endif
+  if (fmt == FGFP8_SCALE_F32) {
+    return wide ? launch_gemm<256, 128, 0, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms)
+                : launch_gemm<128, 64, 0, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms);
+  }
+  return wide ? launch_gemm<256, 128, 1, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms)
+              : launch_gemm<128, 64, 1, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms);
 }
 
 // Few-token (M <= 64) launch: one CTA per 128 output columns, operands swapped.
@@ -182,21 +209,6 @@ fgfp8_status dispatch_decode(const uint8_t* Xq, const void* Xs, int64_t ld_s, co
   if (M <= 16) return launch_decode<16, FMT>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev);
   if (M <= 32) return launch_decode<32, FMT>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev);
   return launch_decode<64, FMT>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev);
-}
-
-template <bool kGrouped>
-fgfp8_status dispatch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws, void* Y,
-                           int64_t M, int64_t N, int64_t K, int fmt, const int32_t* offs, int E, int64_t b_rows,
-                           cudaStream_t s, int dev) {
-  // 256-wide tiles halve the promotion work per MMA; 128-wide ones when N is
-  // not a multiple of 256 or when there are few rows (more CTAs in flight).
-  const bool wide = (N % 256 == 0) && M > 128;
-  if (fmt == FGFP8_SCALE_F32) {
-    return wide ? launch_gemm<256, 0, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev)
-                : launch_gemm<128, 0, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev);
-  }
-  return wide ? launch_gemm<256, 1, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev)
-              : launch_gemm<128, 1, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev);
 }
 
 fgfp8_status check_gemm_common(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
@@ -245,9 +257,9 @@ fgfp8_status fgfp8_quant_act(const void* X, int64_t M, int64_t K, int64_t ldx, u
   st = current_device(&dev, &info);
   if (st != FGFP8_OK) return st;
 
-  constexpr int kUnroll = 2;
+  constexpr int kUnroll = 2;                 // groups in flight per 8-lane group (4 x 16-byte loads per lane)
   const uint64_t groups = static_cast<uint64_t>(M) * (K / 128);
-  const uint64_t want = (groups * 16 + 256 * kUnroll - 1) / (256 * kUnroll);
+  const uint64_t want = (groups * 8 + 256 * kUnroll - 1) / (256 * kUnroll);
   const uint64_t cap = static_cast<uint64_t>(info.sm_count) * 8;
   const unsigned blocks = static_cast<unsigned>(want < cap ? (want ? want : 1) : cap);
   fgfp8::FastDiv kbd(static_cast<uint32_t>(K / 128));
@@ -312,7 +324,7 @@ fgfp8_status fgfp8_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const u
     return fmt == FGFP8_SCALE_F32 ? dispatch_decode<0>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev)
                                   : dispatch_decode<1>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev);
   }
-  return dispatch_gemm<false>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, fmt, nullptr, 1, N, s, dev);
+  return dispatch_gemm<false>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, fmt, nullptr, 1, N, s, dev, info.sm_count);
 }
 
 fgfp8_status fgfp8_grouped_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
@@ -332,7 +344,7 @@ fgfp8_status fgfp8_grouped_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s,
   st = current_device(&dev, &info);
   if (st != FGFP8_OK) return st;
   return dispatch_gemm<true>(Xq, Xs, ld_s, Wq, Ws, Y, M_total, N, K, fmt, group_offs, E,
-                             static_cast<int64_t>(E) * N, reinterpret_cast<cudaStream_t>(stream), dev);
+                             static_cast<int64_t>(E) * N, reinterpret_cast<cudaStream_t>(stream), dev, info.sm_count);
 }
 
 fgfp8_status fgfp8_check_device_status(void* stream) {

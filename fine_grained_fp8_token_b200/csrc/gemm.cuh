@@ -39,20 +39,38 @@ __device__ int g_device_status;
 
 __device__ __forceinline__ void record_status(int code) { atomicCAS(&g_device_status, 0, code); }
 
-template <int BN>
+// Tile configuration of the dense / grouped kernel.  BN: output columns per
+// tile; CW: columns per promotion warp (each warp owns 32 rows x CW columns).
+template <int BN, int CW>
 struct GemmCfg {
   static constexpr int kBM = 128;
   static constexpr int kBK = 128;
-  static constexpr int kStages = (BN == 256) ? 4 : 6;
-  static constexpr int kEpiWarps = BN / 32;                  // one warp per 32 rows x 128 columns
-  static constexpr int kThreads = (2 + kEpiWarps) * 32;
-  static constexpr uint32_t kTmemCols = 2 * BN;              // two partial buffers
+  static constexpr int kEpiWarps = 4 * (BN / CW);
+  static constexpr int kThreads = 128 + kEpiWarps * 32;          // warpgroup 0: producer, MMA, 2 idle
+  static constexpr int kNumBuf = (512 / BN) > 4 ? 4 : (512 / BN);  // TMEM partial buffers
+  static constexpr uint32_t kTmemCols = kNumBuf * BN;
   static constexpr uint32_t kABytes = kBM * kBK;
   static constexpr uint32_t kBBytes = BN * kBK;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = (224 * 1024) / kStageBytes;       // 7 (BN=128) or 4 (BN=256)
   static constexpr size_t kBarrierBytes = 256;
   static constexpr size_t kSmemBytes = 1024 + kStages * static_cast<size_t>(kStageBytes) + kBarrierBytes;
+  // 128 accumulators per thread need more than the launch share of
+  // registers: warpgroup 0 gives some back (setmaxnreg) to the promotion
+  // warpgroups.  launch: 384 threads x 168 = 64512; after: 128 x 40 + 256 x 232.
+  static constexpr bool kRegSplit = CW > 64;
+  static constexpr int kRegsLow = 40;
+  static constexpr int kRegsHigh = 232;
 };
+
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
 
 // Combined block scale sa[m, kb] * sw[nb, kb] for one K block.  fp32 scales
 // multiply in fp32; UE8M0 scales are exponent bytes: 2^(ea-127) * 2^(eb-127)
@@ -113,23 +131,23 @@ __device__ __forceinline__ void produce_tiles(const CUtensorMap* tmA, int a_row,
 }
 
 // MMA issuer (one thread): per K block, four K=32 tcgen05.mma (M=128, N=kN)
-// into TMEM partial buffer kb & 1 (columns [b*kN, b*kN + kN)), overwriting it
-// on the first step; then frees the smem slot and publishes the buffer.  The
-// buffer is reused only after the promotion warps released it.  A final
-// commit makes every MMA complete before the caller may free TMEM.
-template <int kStages, uint32_t kABytes, uint32_t kBBytes, int kN>
+// into TMEM partial buffer kb % kNumBuf (columns [b*kN, b*kN + kN)),
+// overwriting it on the first step; then frees the smem slot and publishes
+// the buffer.  A buffer is reused only after the promotion warps released it.
+// A final commit makes every MMA complete before the caller may free TMEM.
+template <int kStages, uint32_t kABytes, uint32_t kBBytes, int kN, int kNumBuf>
 __device__ __forceinline__ void issue_mmas(uint32_t a_base, uint32_t b_base, int KB, uint32_t tmem_base,
                                            uint64_t* full, uint64_t* empty, uint64_t* tfull, uint64_t* tempty,
                                            uint64_t* mma_done) {
   constexpr uint32_t idesc = idesc_e4m3_f32(128, kN);
   for (int kb = 0; kb < KB; ++kb) {
     const int s = kb % kStages;
-    const int b = kb & 1;
+    const int b = kb % kNumBuf;
     if (!mbar_wait(&full[s], (kb / kStages) & 1u)) {
       record_status(kDevTimeoutMma);
       break;
     }
-    if (kb >= 2 && !mbar_wait(&tempty[b], ((kb >> 1) & 1u) ^ 1u)) {
+    if (kb >= kNumBuf && !mbar_wait(&tempty[b], ((kb / kNumBuf) & 1u) ^ 1u)) {
       record_status(kDevTimeoutMma);
       break;
     }
@@ -148,13 +166,13 @@ __device__ __forceinline__ void issue_mmas(uint32_t a_base, uint32_t b_base, int
   if (!mbar_wait(mma_done, 0)) record_status(kDevTimeoutMma);
 }
 
-template <int BN, int FMT, bool kGrouped>
-__global__ void __launch_bounds__(GemmCfg<BN>::kThreads, 1)
+template <int BN, int CW, int FMT, bool kGrouped>
+__global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
     gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const void* __restrict__ Xs, uint32_t ld_s, const void* __restrict__ Ws,
                             __nv_bfloat16* __restrict__ Y, int M, int N, int K,
-                            const int32_t* __restrict__ group_offs, int E) {
-  using C = GemmCfg<BN>;
+                            const int32_t* __restrict__ group_offs, int E, int num_tiles) {
+  using C = GemmCfg<BN, CW>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -162,44 +180,40 @@ __global__ void __launch_bounds__(GemmCfg<BN>::kThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::kStages * C::kBBytes);
   uint64_t* empty = full + C::kStages;
   uint64_t* tfull = empty + C::kStages;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* mma_done = tempty + 2;
+  uint64_t* tempty = tfull + C::kNumBuf;
+  uint64_t* mma_done = tempty + C::kNumBuf;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int KB = K / C::kBK;
   const int NB = N / 128;
+  const int num_m = (M + C::kBM - 1) / C::kBM;
+  const int num_n = N / BN;
 
-  // ---- tile coordinates
-  int m_tile, n_tile;
-  if (!kGrouped) {
-    const int num_m = (M + C::kBM - 1) / C::kBM;
-    m_tile = blockIdx.x % num_m;
-    n_tile = blockIdx.x / num_m;
-  } else {
-    const int num_n = N / BN;
-    n_tile = blockIdx.x % num_n;
-    m_tile = blockIdx.x / num_n;
-  }
-  const int m0 = m_tile * C::kBM;
-  const int n0 = n_tile * BN;
-  int expert = 0;
-  if (kGrouped) {
-    expert = find_expert(group_offs, E, m0);
-    if (expert < 0) {                        // uniform across the CTA
-      if (threadIdx.x == 0) record_status(kDevBadGroupOffsets);
-      return;
+  // Tile t -> (m0, n0, expert).  Dense tiles run M-fastest (the activation
+  // tile set stays L2-resident while a weight tile is reused); grouped tiles
+  // run N-fastest (the CTAs of one expert share its weights in L2).  An
+  // expert of -1 marks a tile whose rows no segment covers: every role skips
+  // it and the status word records it.
+  auto coords = [&](int t, int& m0, int& n0, int& expert) {
+    if (!kGrouped) {
+      m0 = (t % num_m) * C::kBM;
+      n0 = (t / num_m) * BN;
+      expert = 0;
+    } else {
+      n0 = (t % num_n) * BN;
+      m0 = (t / num_n) * C::kBM;
+      expert = find_expert(group_offs, E, m0);
     }
-  }
+  };
 
-  // ---- setup: barriers (thread 0), TMEM (warp 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < C::kNumBuf; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], C::kEpiWarps);
     }
@@ -219,77 +233,142 @@ __global__ void __launch_bounds__(GemmCfg<BN>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
-    // ================= TMA producer
-    if (lane == 0)
-      produce_tiles<C::kStages, C::kABytes, C::kBBytes>(&tmA, m0, &tmB, expert * N + n0, KB, sA, sB, full, empty);
-  } else if (warp == 1) {
-    // ================= MMA issuer
-    if (lane == 0)
-      issue_mmas<C::kStages, C::kABytes, C::kBBytes, BN>(smem_u32(sA), smem_u32(sB), KB, tmem_base, full, empty,
-                                                         tfull, tempty, mma_done);
-  } else {
-    // ================= promotion / epilogue
-    const int ew = warp - 2;
-    const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
-    const int col0 = (ew >> 2) * 128;          // column half (BN = 256) or 0
-    const int row = quad * 32 + lane;
-    const int m = m0 + row;
-    const bool row_ok = m < M;
-    const bool col_ok = n0 + col0 < N;
-    const uint64_t ws_row = (static_cast<uint64_t>(expert) * NB + (n0 + col0) / 128) * KB;
-    const uint32_t taddr0 = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(col0);
-
-    float acc[128];
-#pragma unroll
-    for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
-
-    auto scale_of = [&](int kb) -> float {
-      return (row_ok && col_ok) ? block_scale<FMT>(Xs, static_cast<uint64_t>(kb) * ld_s + m, Ws, ws_row + kb)
-                                : 0.0f;
-    };
-
-    bool ok = true;
-    float s_next = scale_of(0);
-    for (int kb = 0; kb < KB; ++kb) {
-      const int b = kb & 1;
-      const float s = s_next;
-      if (kb + 1 < KB) s_next = scale_of(kb + 1);
-      // the outcome is made warp-uniform: the TMEM loads below are .sync.aligned
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[b], (kb >> 1) & 1u))) {
-        if (lane == 0) record_status(kDevTimeoutEpilogue);
-        ok = false;
-        break;
+  if (warp < 4) {
+    if (C::kRegSplit) setmaxnreg_dec<C::kRegsLow>();
+    if (warp == 0 && lane == 0) {
+      // ================= TMA producer
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        int m0, n0, expert;
+        coords(t, m0, n0, expert);
+        if (expert < 0) {
+          record_status(kDevBadGroupOffsets);
+          continue;
+        }
+        const int b_row = expert * N + n0;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % C::kStages;
+          if (it >= static_cast<uint32_t>(C::kStages) && !mbar_wait(&empty[s], ((it / C::kStages) & 1u) ^ 1u)) {
+            record_status(kDevTimeoutProducer);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+          tma_load_2d(sA + s * C::kABytes, &tmA, &full[s], kb * C::kBK, m0);
+          tma_load_2d(sB + s * C::kBBytes, &tmB, &full[s], kb * C::kBK, b_row);
+        }
       }
-      tc_fence_after();
-      const uint32_t taddr = taddr0 + static_cast<uint32_t>(b * BN);
+      // every copy issued must land before the CTA may exit
+      for (uint32_t j = (it > static_cast<uint32_t>(C::kStages) ? it - C::kStages : 0); j < it; ++j)
+        if (!mbar_wait(&full[j % C::kStages], (j / C::kStages) & 1u)) record_status(kDevTimeoutProducer);
+    } else if (warp == 1 && lane == 0) {
+      // ================= MMA issuer
+      constexpr uint32_t idesc = idesc_e4m3_f32(128, BN);
+      const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
+      uint32_t it = 0, bt = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        int m0, n0, expert;
+        coords(t, m0, n0, expert);
+        if (expert < 0) continue;
+        for (int kb = 0; kb < KB; ++kb, ++it, ++bt) {
+          const int s = it % C::kStages;
+          const int buf = bt % C::kNumBuf;
+          if (!mbar_wait(&full[s], (it / C::kStages) & 1u)) {
+            record_status(kDevTimeoutMma);
+            ok = false;
+            break;
+          }
+          if (bt >= static_cast<uint32_t>(C::kNumBuf) &&
+              !mbar_wait(&tempty[buf], ((bt / C::kNumBuf) & 1u) ^ 1u)) {
+            record_status(kDevTimeoutMma);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t p[32];
-        tmem_ld_32x32b_x32(taddr + c * 32, p);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) acc[c * 32 + j] = __fmaf_rn(__uint_as_float(p[j]), s, acc[c * 32 + j]);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = smem_desc_k_sw128(a_base + s * C::kABytes + kk * 32);
+            const uint64_t bd = smem_desc_k_sw128(b_base + s * C::kBBytes + kk * 32);
+            mma_f8f6f4(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&empty[s]);
+          mma_commit(&tfull[buf]);
+        }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[b]);
+      mma_commit(mma_done);
+      if (!mbar_wait(mma_done, 0)) record_status(kDevTimeoutMma);
     }
+  } else {
+    if (C::kRegSplit) setmaxnreg_inc<C::kRegsHigh>();
+    // ================= promotion / epilogue
+    const int ew = warp - 4;
+    const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
+    const int col0 = (ew >> 2) * CW;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(col0);
+    uint32_t bt = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      int m0, n0, expert;
+      coords(t, m0, n0, expert);
+      if (expert < 0) continue;
+      const int m = m0 + row;
+      const bool live = (m < M) && (n0 + col0 < N);
+      const uint64_t ws_row = (static_cast<uint64_t>(expert) * NB + (n0 + col0) / 128) * KB;
+      auto scale_of = [&](int kb) -> float {
+        return live ? block_scale<FMT>(Xs, static_cast<uint64_t>(kb) * ld_s + m, Ws, ws_row + kb) : 0.0f;
+      };
 
-    if (ok && row_ok && col_ok) {
-      __nv_bfloat16* yrow = Y + static_cast<uint64_t>(m) * N + n0 + col0;
+      float acc[CW];
 #pragma unroll
-      for (int j = 0; j < 128; j += 8) {
-        uint4 v;
-        __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[j + 0], acc[j + 1]);
-        __nv_bfloat162 h1 = __floats2bfloat162_rn(acc[j + 2], acc[j + 3]);
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[j + 4], acc[j + 5]);
-        __nv_bfloat162 h3 = __floats2bfloat162_rn(acc[j + 6], acc[j + 7]);
-        v.x = *reinterpret_cast<uint32_t*>(&h0);
-        v.y = *reinterpret_cast<uint32_t*>(&h1);
-        v.z = *reinterpret_cast<uint32_t*>(&h2);
-        v.w = *reinterpret_cast<uint32_t*>(&h3);
-        *reinterpret_cast<uint4*>(yrow + j) = v;
+      for (int j = 0; j < CW; ++j) acc[j] = 0.0f;
+      float s_next = scale_of(0);
+      for (int kb = 0; kb < KB; ++kb, ++bt) {
+        const int buf = bt % C::kNumBuf;
+        const float sc = s_next;
+        if (kb + 1 < KB) s_next = scale_of(kb + 1);
+        // warp-uniform outcome: the TMEM loads below are .sync.aligned
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[buf], (bt / C::kNumBuf) & 1u))) {
+          if (lane == 0) record_status(kDevTimeoutEpilogue);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t taddr = lane_base + static_cast<uint32_t>(buf * BN);
+#pragma unroll
+        for (int h = 0; h < CW / 64; ++h) {
+          uint32_t p0[32], p1[32];
+          tmem_ld_32x32b_x32(taddr + h * 64, p0);
+          tmem_ld_32x32b_x32(taddr + h * 64 + 32, p1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) acc[h * 64 + j] = __fmaf_rn(__uint_as_float(p0[j]), sc, acc[h * 64 + j]);
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            acc[h * 64 + 32 + j] = __fmaf_rn(__uint_as_float(p1[j]), sc, acc[h * 64 + 32 + j]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[buf]);
+      }
+      if (ok && live) {
+        __nv_bfloat16* yrow = Y + static_cast<uint64_t>(m) * N + n0 + col0;
+#pragma unroll
+        for (int j = 0; j < CW; j += 8) {
+          uint4 v;
+          __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[j + 0], acc[j + 1]);
+          __nv_bfloat162 h1 = __floats2bfloat162_rn(acc[j + 2], acc[j + 3]);
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[j + 4], acc[j + 5]);
+          __nv_bfloat162 h3 = __floats2bfloat162_rn(acc[j + 6], acc[j + 7]);
+          v.x = *reinterpret_cast<uint32_t*>(&h0);
+          v.y = *reinterpret_cast<uint32_t*>(&h1);
+          v.z = *reinterpret_cast<uint32_t*>(&h2);
+          v.w = *reinterpret_cast<uint32_t*>(&h3);
+          *reinterpret_cast<uint4*>(yrow + j) = v;
+        }
       }
     }
   }
@@ -300,7 +379,6 @@ __global__ void __launch_bounds__(GemmCfg<BN>::kThreads, 1)
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
 }
-
 
 // ---------------------------------------------------------------------------
 // Few-token variant (M <= 64, decode): operands swapped so the weight supplies
@@ -318,7 +396,8 @@ struct DecodeCfg {
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
   static constexpr int kStages = (200 * 1024) / kStageBytes > 12 ? 12 : (200 * 1024) / kStageBytes;
   static constexpr int kThreads = 6 * 32;                    // producer, MMA, 4 promotion warps
-  static constexpr uint32_t kTmemCols = (2 * BNT < 32) ? 32 : 2 * BNT;
+  static constexpr int kNumBuf = 4;                          // TMEM partial buffers
+  static constexpr uint32_t kTmemCols = (kNumBuf * BNT < 32) ? 32 : kNumBuf * BNT;
   static constexpr size_t kSmemBytes = 1024 + kStages * static_cast<size_t>(kStageBytes) + 256;
 };
 
@@ -350,8 +429,8 @@ __global__ void __launch_bounds__(DecodeCfg<BNT>::kThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(sX + C::kStages * C::kBBytes);
   uint64_t* empty = full + C::kStages;
   uint64_t* tfull = empty + C::kStages;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* mma_done = tempty + 2;
+  uint64_t* tempty = tfull + C::kNumBuf;
+  uint64_t* mma_done = tempty + C::kNumBuf;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -364,7 +443,7 @@ __global__ void __launch_bounds__(DecodeCfg<BNT>::kThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < C::kNumBuf; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], 4);
     }
@@ -389,8 +468,8 @@ __global__ void __launch_bounds__(DecodeCfg<BNT>::kThreads, 1)
       produce_tiles<C::kStages, C::kABytes, C::kBBytes>(&tmW, n0, &tmX, 0, KB, sW, sX, full, empty);
   } else if (warp == 1) {
     if (lane == 0)
-      issue_mmas<C::kStages, C::kABytes, C::kBBytes, BNT>(smem_u32(sW), smem_u32(sX), KB, tmem_base, full, empty,
-                                                          tfull, tempty, mma_done);
+      issue_mmas<C::kStages, C::kABytes, C::kBBytes, BNT, C::kNumBuf>(smem_u32(sW), smem_u32(sX), KB, tmem_base,
+                                                                      full, empty, tfull, tempty, mma_done);
   } else {
     const int quad = warp & 3;
     const int n = n0 + quad * 32 + lane;
@@ -402,45 +481,41 @@ __global__ void __launch_bounds__(DecodeCfg<BNT>::kThreads, 1)
 #pragma unroll
     for (int j = 0; j < BNT; ++j) acc[j] = 0.0f;
 
-    // raw scales of block kb: lane l holds the token scales l, l+32 (if < M)
-    auto load_scales = [&](int kb, uint32_t (&sa)[kT], uint32_t& sw) {
+    // combined scales of block kb: lane l holds sa[l]*sw and sa[l+32]*sw
+    // (0 for tokens >= M); column c then takes lane c%32 of word c/32
+    auto scales_of = [&](int kb, float (&sc)[kT]) {
+      const uint32_t sw = load_scale_raw<FMT>(Ws, ws_row + kb);
 #pragma unroll
       for (int t = 0; t < kT; ++t) {
         const int m = t * 32 + lane;
-        sa[t] = m < M ? load_scale_raw<FMT>(Xs, static_cast<uint64_t>(kb) * ld_s + m) : 0u;
+        sc[t] = m < M ? combine_raw<FMT>(load_scale_raw<FMT>(Xs, static_cast<uint64_t>(kb) * ld_s + m), sw) : 0.0f;
       }
-      sw = load_scale_raw<FMT>(Ws, ws_row + kb);
     };
 
     bool ok = true;
-    uint32_t sa_next[kT], sw_next;
-    load_scales(0, sa_next, sw_next);
+    float sc_next[kT];
+    scales_of(0, sc_next);
     for (int kb = 0; kb < KB; ++kb) {
-      const int b = kb & 1;
-      uint32_t sa[kT];
+      const int b = kb % C::kNumBuf;
+      float sc[kT];
 #pragma unroll
-      for (int t = 0; t < kT; ++t) sa[t] = sa_next[t];
-      const uint32_t sw = sw_next;
-      if (kb + 1 < KB) load_scales(kb + 1, sa_next, sw_next);
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[b], (kb >> 1) & 1u))) {
+      for (int t = 0; t < kT; ++t) sc[t] = sc_next[t];
+      if (kb + 1 < KB) scales_of(kb + 1, sc_next);
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[b], (kb / C::kNumBuf) & 1u))) {
         if (lane == 0) record_status(kDevTimeoutEpilogue);
         ok = false;
         break;
       }
       tc_fence_after();
       const uint32_t taddr = taddr0 + static_cast<uint32_t>(b * BNT);
+      uint32_t p[BNT];
 #pragma unroll
-      for (int c = 0; c < BNT / 16; ++c) {
-        uint32_t p[16];
-        tmem_ld_32x32b_x16(taddr + c * 16, p);
-        tmem_wait_ld();
+      for (int c = 0; c < BNT / 16; ++c) tmem_ld_32x32b_x16(taddr + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&p[c * 16]));
+      tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int m = c * 16 + j;
-          const uint32_t a = __shfl_sync(0xFFFFFFFFu, sa[m / 32], m % 32);
-          const float sc = (m < M) ? combine_raw<FMT>(a, sw) : 0.0f;
-          acc[m] = __fmaf_rn(__uint_as_float(p[j]), sc, acc[m]);
-        }
+      for (int m = 0; m < BNT; ++m) {
+        const float a = __shfl_sync(0xFFFFFFFFu, sc[m / 32], m % 32);
+        acc[m] = __fmaf_rn(__uint_as_float(p[m]), a, acc[m]);
       }
       tc_fence_before();
       __syncwarp();

@@ -7,14 +7,16 @@
 //   fp32  : s = amax / 448 (IEEE division), code = E4M3_rne_satfinite(x / s)
 //   UE8M0 : s = 2^ceil(log2(amax / 448)), stored as its biased exponent byte
 //
-// x / s is evaluated without a per-element division: with r = RN(1/s),
-// q0 = RN(|x| r), e = fma(-q0, s, |x|), q = fma(e, r, q0) is the correctly
-// rounded quotient (Markstein's theorem, "IA-64 and Elementary Functions",
-// 2000; Muller et al., "Handbook of Floating-Point Arithmetic", the FMA-based
-// division section).  A host-side test checks it against IEEE division on
-// every (bf16 element, bf16 amax) pair the kernel can meet.  For UE8M0 the
-// quotient is |x| * 2^-p, exact.  The sign of x is applied to the E4M3 code
-// afterwards, so -0 and tiny negatives keep it.
+// Divisions are evaluated without a division routine: with r = RN(1/d),
+// q0 = RN(a r), e = fma(-q0, d, a), q = fma(e, r, q0) is the correctly
+// rounded a/d (Markstein's theorem, "IA-64 and Elementary Functions", 2000;
+// Muller et al., "Handbook of Floating-Point Arithmetic", the FMA-based
+// division section).  It is used for amax/448 (r = RN(1/448), a constant) and
+// for |x|/s (r = RN(1/s) once per group).  A host-side test checks both
+// against IEEE division on every input the kernel can meet: every bf16 amax,
+// and every (bf16 element, bf16 amax) pair.  For UE8M0 the quotient is
+// |x| * 2^-p, exact.  The sign of x is applied to the E4M3 code afterwards,
+// so -0 and tiny negatives keep it.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
@@ -70,9 +72,11 @@ struct GroupScale {
 
 template <int FMT>
 __device__ __forceinline__ GroupScale make_scale(uint32_t amax_bits) {
-  float amax = __uint_as_float(amax_bits << 16);
-  float amax_c = amax < 1e-4f ? 1e-4f : amax;          // NaN stays NaN
-  float t = __fdiv_rn(amax_c, 448.0f);
+  const float amax = __uint_as_float(amax_bits << 16);
+  const float amax_c = amax < 1e-4f ? 1e-4f : amax;    // NaN stays NaN
+  constexpr float kR448 = 1.0f / 448.0f;               // RN(1/448), folded at compile time
+  const float q0 = __fmul_rn(amax_c, kR448);
+  const float t = __fmaf_rn(__fmaf_rn(-q0, 448.0f, amax_c), kR448, q0);   // = RN(amax_c / 448)
   GroupScale g;
   if (FMT == 0) {
     g.s = t;
@@ -89,40 +93,44 @@ __device__ __forceinline__ GroupScale make_scale(uint32_t amax_bits) {
   return g;
 }
 
-// |x|/s for the magnitude bits `h` (bf16 without sign) of one element.
+// |x|/s for one element, x given as an fp32 (its bf16 bits in the top half).
 template <int FMT>
-__device__ __forceinline__ float quotient(uint32_t h, const GroupScale& g) {
-  float a = __uint_as_float(h << 16);
+__device__ __forceinline__ float quotient(float x, const GroupScale& g) {
+  const float a = fabsf(x);
   if (FMT == 0) {
-    float q0 = __fmul_rn(a, g.r);
-    float e = __fmaf_rn(-q0, g.s, a);
+    const float q0 = __fmul_rn(a, g.r);
+    const float e = __fmaf_rn(-q0, g.s, a);
     return __fmaf_rn(e, g.r, q0);
   } else {
     return __fmul_rn(a, g.r);
   }
 }
 
-// Two packed bf16 (w) -> two E4M3 codes in the low 16 bits (element 0 low).
+// Four bf16 (two packed words) -> four E4M3 codes in one word (element 0 in
+// the low byte).  Magnitudes are quantized; the four sign bits (bit 7 of the
+// bf16 bytes 1 and 3 of each word) are gathered with one byte permute.
 template <int FMT>
-__device__ __forceinline__ uint32_t quant_pair(uint32_t w, const GroupScale& g) {
-  float q_lo = quotient<FMT>(w & 0x7FFFu, g);
-  float q_hi = quotient<FMT>((w >> 16) & 0x7FFFu, g);
-  uint32_t c = __nv_cvt_float2_to_fp8x2(make_float2(q_lo, q_hi), __NV_SATFINITE, __NV_E4M3);
-  return (c & 0xFFFFu) | ((w >> 8) & 0x80u) | ((w >> 16) & 0x8000u);
+__device__ __forceinline__ uint32_t quant4(uint32_t w0, uint32_t w1, const GroupScale& g) {
+  const uint32_t c0 = __nv_cvt_float2_to_fp8x2(
+      make_float2(quotient<FMT>(__uint_as_float(w0 << 16), g), quotient<FMT>(__uint_as_float(w0 & 0xFFFF0000u), g)),
+      __NV_SATFINITE, __NV_E4M3);
+  const uint32_t c1 = __nv_cvt_float2_to_fp8x2(
+      make_float2(quotient<FMT>(__uint_as_float(w1 << 16), g), quotient<FMT>(__uint_as_float(w1 & 0xFFFF0000u), g)),
+      __NV_SATFINITE, __NV_E4M3);
+  const uint32_t codes = __byte_perm(c0, c1, 0x5410);
+  const uint32_t signs = __byte_perm(w0, w1, 0x7531) & 0x80808080u;
+  return codes | signs;
 }
 
 template <int FMT>
 __device__ __forceinline__ uint2 quant8(const uint4& v, const GroupScale& g) {
-  uint2 out;
-  out.x = quant_pair<FMT>(v.x, g) | (quant_pair<FMT>(v.y, g) << 16);
-  out.y = quant_pair<FMT>(v.z, g) | (quant_pair<FMT>(v.w, g) << 16);
-  return out;
+  return make_uint2(quant4<FMT>(v.x, v.y, g), quant4<FMT>(v.z, v.w, g));
 }
 
 // ---------------------------------------------------------------------------
-// Activation quantization.  One half-warp per 128-element group (16 lanes x
-// 16 bytes), UNROLL groups in flight per half-warp, grid-stride over the
-// M*K/128 groups in row-major order.
+// Activation quantization.  Eight lanes per 128-element group, 16 elements
+// (two 16-byte loads) per lane, UNROLL groups in flight per lane group,
+// grid-stride over the M*K/128 groups in row-major order.
 // X bf16 [M, K] row stride ldx  ->  Xq u8 [M, K] row stride K,
 // scales Xs[g * ld_s + m] (fp32 or UE8M0 byte).
 // ---------------------------------------------------------------------------
@@ -132,33 +140,39 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
                                                         void* __restrict__ Xs, uint64_t ld_s, FastDiv kb_div) {
   const uint32_t total = M * kb_div.d;
   const uint32_t lane = threadIdx.x & 31u;
-  const uint32_t sub = lane & 15u;
-  const uint32_t hmask = 0xFFFFu << (lane & 16u);
-  const uint32_t hw = (blockIdx.x * blockDim.x + threadIdx.x) >> 4;
-  const uint32_t nhw = (gridDim.x * blockDim.x) >> 4;
+  const uint32_t sub = lane & 7u;
+  const uint32_t gmask = 0xFFu << (lane & 24u);            // the 8 lanes sharing a group
+  const uint32_t grp = (blockIdx.x * blockDim.x + threadIdx.x) >> 3;
+  const uint32_t ngrp = (gridDim.x * blockDim.x) >> 3;
 
-  for (uint32_t base = hw; base < total; base += nhw * UNROLL) {
-    uint4 v[UNROLL];
+  for (uint32_t base = grp; base < total; base += ngrp * UNROLL) {
+    uint4 v[UNROLL][2];
     uint32_t m[UNROLL], g[UNROLL];
 #pragma unroll
     for (int u = 0; u < UNROLL; ++u) {
-      const uint32_t gi = base + u * nhw;
+      const uint32_t gi = base + u * ngrp;
       if (gi < total) {
         m[u] = kb_div.div(gi);
         g[u] = gi - m[u] * kb_div.d;
-        v[u] = ld_stream_v4(X + m[u] * ldx + g[u] * kGroup + sub * 8u);
+        const uint16_t* src = X + m[u] * ldx + g[u] * kGroup + sub * 16u;
+        v[u][0] = ld_stream_v4(src);
+        v[u][1] = ld_stream_v4(src + 8);
       }
     }
 #pragma unroll
     for (int u = 0; u < UNROLL; ++u) {
-      const uint32_t gi = base + u * nhw;
+      const uint32_t gi = base + u * ngrp;
       if (gi < total) {
-        uint32_t a = absmax_bits8(v[u]);
+        uint32_t a = max(absmax_bits8(v[u][0]), absmax_bits8(v[u][1]));
 #pragma unroll
-        for (int o = 8; o > 0; o >>= 1) a = max(a, __shfl_xor_sync(hmask, a, o));
+        for (int o = 4; o > 0; o >>= 1) a = max(a, __shfl_xor_sync(gmask, a, o));
         const GroupScale gs = make_scale<FMT>(a);
-        const uint2 codes = quant8<FMT>(v[u], gs);
-        *reinterpret_cast<uint2*>(Xq + static_cast<uint64_t>(m[u]) * K + g[u] * kGroup + sub * 8u) = codes;
+        uint4 codes;
+        codes.x = quant4<FMT>(v[u][0].x, v[u][0].y, gs);
+        codes.y = quant4<FMT>(v[u][0].z, v[u][0].w, gs);
+        codes.z = quant4<FMT>(v[u][1].x, v[u][1].y, gs);
+        codes.w = quant4<FMT>(v[u][1].z, v[u][1].w, gs);
+        *reinterpret_cast<uint4*>(Xq + static_cast<uint64_t>(m[u]) * K + g[u] * kGroup + sub * 16u) = codes;
         if (sub == 0) {
           const uint64_t si = static_cast<uint64_t>(g[u]) * ld_s + m[u];
           if (FMT == 0) reinterpret_cast<float*>(Xs)[si] = gs.s;

@@ -73,5 +73,22 @@ int main() {
     }
   }
   std::printf("quotient pairs: %ld (of which %ld both <= 2^-10) mismatches: %ld\n", pairs, below, qbad);
-  return qbad ? 2 : 0;
+  if (qbad) return 2;
+
+  // ---- 3. amax / 448 by the same FMA-based division with the constant
+  //         r448 = RN(1/448), against IEEE division, for every positive bf16
+  //         amax (finite and infinite) and the 1e-4 floor
+  const float r448 = 1.0f / 448.0f;
+  long sbad = 0;
+  for (uint32_t ab = 1; ab <= 0x7F80; ++ab) {
+    const float amax = bf16_bits_to_float(ab);
+    const float a = amax < 1e-4f ? 1e-4f : amax;
+    const float q0 = a * r448;
+    const float e = std::fmaf(-q0, 448.0f, a);
+    const float q = std::fmaf(e, r448, q0);
+    const float ref = a / 448.0f;
+    if (fbits(q) != fbits(ref) && !(std::isinf(ref) && std::isnan(q))) ++sbad;
+  }
+  std::printf("scale divisions checked: %u mismatches: %ld\n", 0x7F80u, sbad);
+  return sbad ? 3 : 0;
 }
