@@ -57,9 +57,9 @@ struct GemmCfg {
   static constexpr size_t kSmemBytes = 1024 + kStages * static_cast<size_t>(kStageBytes) + kBarrierBytes;
   // 128 accumulators per thread need more than the launch share of
   // registers: warpgroup 0 gives some back (setmaxnreg) to the promotion
-  // warpgroups.  launch: 384 threads x 168 = 64512; after: 128 x 40 + 256 x 232.
+  // warpgroups.  launch: 384 threads x 168 = 64512; after: 128 x 32 + 256 x 232.
   static constexpr bool kRegSplit = CW > 64;
-  static constexpr int kRegsLow = 40;
+  static constexpr int kRegsLow = 32;
   static constexpr int kRegsHigh = 232;
 };
 
@@ -72,21 +72,29 @@ __device__ __forceinline__ void setmaxnreg_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
-// Combined block scale sa[m, kb] * sw[nb, kb] for one K block.  fp32 scales
-// multiply in fp32; UE8M0 scales are exponent bytes: 2^(ea-127) * 2^(eb-127)
-// = 2^(ea+eb-254), built exactly from the biased exponent ea+eb-127 (or by
-// ldexpf when that leaves the normal range).  A 0xFF (NaN) scale byte gives
-// an unspecified product.
+// Block scales travel as raw 32-bit words (fp32 bits, or a UE8M0 byte) from
+// their load until the K block that uses them, so the loads can be issued
+// several K blocks ahead without stalling on them; combine_raw then forms
+// sa[m, kb] * sw[nb, kb]: an fp32 product, or for UE8M0 exponent bytes
+// 2^(ea-127) * 2^(eb-127) = 2^(ea+eb-254) built exactly from the biased
+// exponent ea+eb-127 (ldexpf when that leaves the normal range).  A 0xFF
+// (NaN) scale byte gives an unspecified product.
 template <int FMT>
-__device__ __forceinline__ float block_scale(const void* __restrict__ Xs, uint64_t ia, const void* __restrict__ Ws,
-                                             uint64_t iw) {
-  if (FMT == 0) return __ldg(reinterpret_cast<const float*>(Xs) + ia) * __ldg(reinterpret_cast<const float*>(Ws) + iw);
-  const int ea = __ldg(reinterpret_cast<const uint8_t*>(Xs) + ia);
-  const int eb = __ldg(reinterpret_cast<const uint8_t*>(Ws) + iw);
-  const int e = ea + eb - 127;
-  if (e >= 1 && e <= 254) return __int_as_float(e << 23);
-  return ldexpf(1.0f, ea + eb - 254);
+__device__ __forceinline__ uint32_t load_scale_raw(const void* __restrict__ p, uint64_t i) {
+  if (FMT == 0) return __float_as_uint(__ldg(reinterpret_cast<const float*>(p) + i));
+  return __ldg(reinterpret_cast<const uint8_t*>(p) + i);
 }
+
+template <int FMT>
+__device__ __forceinline__ float combine_raw(uint32_t a, uint32_t w) {
+  if (FMT == 0) return __uint_as_float(a) * __uint_as_float(w);
+  const int e = static_cast<int>(a) + static_cast<int>(w) - 127;
+  if (e >= 1 && e <= 254) return __int_as_float(e << 23);
+  return ldexpf(1.0f, static_cast<int>(a) + static_cast<int>(w) - 254);
+}
+
+// Depth (in K blocks) of the scale prefetch ring of the promotion warps.
+constexpr int kScaleAhead = 4;
 
 // Expert owning row m: the e with offs[e] <= m < offs[e+1] (binary search),
 // or -1 when the offsets are inconsistent with m.
@@ -318,41 +326,56 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
       const int m = m0 + row;
       const bool live = (m < M) && (n0 + col0 < N);
       const uint64_t ws_row = (static_cast<uint64_t>(expert) * NB + (n0 + col0) / 128) * KB;
-      auto scale_of = [&](int kb) -> float {
-        return live ? block_scale<FMT>(Xs, static_cast<uint64_t>(kb) * ld_s + m, Ws, ws_row + kb) : 0.0f;
+      // raw scale words for K blocks kb .. kb+kScaleAhead-1, ring slot kb % kScaleAhead
+      uint32_t ra[kScaleAhead], rw[kScaleAhead];
+      auto fetch = [&](int kb, uint32_t& a, uint32_t& w) {
+        if (live && kb < KB) {
+          a = load_scale_raw<FMT>(Xs, static_cast<uint64_t>(kb) * ld_s + m);
+          w = load_scale_raw<FMT>(Ws, ws_row + kb);
+        } else {
+          a = 0u;
+          w = 0u;
+        }
       };
+#pragma unroll
+      for (int d = 0; d < kScaleAhead; ++d) fetch(d, ra[d], rw[d]);
 
       float acc[CW];
 #pragma unroll
       for (int j = 0; j < CW; ++j) acc[j] = 0.0f;
-      float s_next = scale_of(0);
-      for (int kb = 0; kb < KB; ++kb, ++bt) {
-        const int buf = bt % C::kNumBuf;
-        const float sc = s_next;
-        if (kb + 1 < KB) s_next = scale_of(kb + 1);
-        // warp-uniform outcome: the TMEM loads below are .sync.aligned
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[buf], (bt / C::kNumBuf) & 1u))) {
-          if (lane == 0) record_status(kDevTimeoutEpilogue);
-          ok = false;
-          break;
+      for (int kb0 = 0; kb0 < KB && ok; kb0 += kScaleAhead) {
+#pragma unroll
+        for (int d = 0; d < kScaleAhead; ++d) {
+          const int kb = kb0 + d;
+          if (kb >= KB) break;
+          const float sc = live ? combine_raw<FMT>(ra[d], rw[d]) : 0.0f;
+          fetch(kb + kScaleAhead, ra[d], rw[d]);
+          const int buf = bt % C::kNumBuf;
+          // warp-uniform outcome: the TMEM loads below are .sync.aligned
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[buf], (bt / C::kNumBuf) & 1u))) {
+            if (lane == 0) record_status(kDevTimeoutEpilogue);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t taddr = lane_base + static_cast<uint32_t>(buf * BN);
+#pragma unroll
+          for (int h = 0; h < CW / 64; ++h) {
+            uint32_t p0[32], p1[32];
+            tmem_ld_32x32b_x32(taddr + h * 64, p0);
+            tmem_ld_32x32b_x32(taddr + h * 64 + 32, p1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc[h * 64 + j] = __fmaf_rn(__uint_as_float(p0[j]), sc, acc[h * 64 + j]);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              acc[h * 64 + 32 + j] = __fmaf_rn(__uint_as_float(p1[j]), sc, acc[h * 64 + 32 + j]);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[buf]);
+          ++bt;
         }
-        tc_fence_after();
-        const uint32_t taddr = lane_base + static_cast<uint32_t>(buf * BN);
-#pragma unroll
-        for (int h = 0; h < CW / 64; ++h) {
-          uint32_t p0[32], p1[32];
-          tmem_ld_32x32b_x32(taddr + h * 64, p0);
-          tmem_ld_32x32b_x32(taddr + h * 64 + 32, p1);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) acc[h * 64 + j] = __fmaf_rn(__uint_as_float(p0[j]), sc, acc[h * 64 + j]);
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            acc[h * 64 + 32 + j] = __fmaf_rn(__uint_as_float(p1[j]), sc, acc[h * 64 + 32 + j]);
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[buf]);
       }
       if (ok && live) {
         __nv_bfloat16* yrow = Y + static_cast<uint64_t>(m) * N + n0 + col0;
@@ -400,21 +423,6 @@ struct DecodeCfg {
   static constexpr uint32_t kTmemCols = (kNumBuf * BNT < 32) ? 32 : kNumBuf * BNT;
   static constexpr size_t kSmemBytes = 1024 + kStages * static_cast<size_t>(kStageBytes) + 256;
 };
-
-template <int FMT>
-__device__ __forceinline__ uint32_t load_scale_raw(const void* __restrict__ p, uint64_t i) {
-  if (FMT == 0) return __float_as_uint(__ldg(reinterpret_cast<const float*>(p) + i));
-  return __ldg(reinterpret_cast<const uint8_t*>(p) + i);
-}
-
-// sa * sw from raw scale words (fp32 bits or UE8M0 bytes).
-template <int FMT>
-__device__ __forceinline__ float combine_raw(uint32_t a, uint32_t w) {
-  if (FMT == 0) return __uint_as_float(a) * __uint_as_float(w);
-  const int e = static_cast<int>(a) + static_cast<int>(w) - 127;
-  if (e >= 1 && e <= 254) return __int_as_float(e << 23);
-  return ldexpf(1.0f, static_cast<int>(a) + static_cast<int>(w) - 254);
-}
 
 template <int BNT, int FMT>
 __global__ void __launch_bounds__(DecodeCfg<BNT>::kThreads, 1)
@@ -481,45 +489,53 @@ __global__ void __launch_bounds__(DecodeCfg<BNT>::kThreads, 1)
 #pragma unroll
     for (int j = 0; j < BNT; ++j) acc[j] = 0.0f;
 
-    // combined scales of block kb: lane l holds sa[l]*sw and sa[l+32]*sw
-    // (0 for tokens >= M); column c then takes lane c%32 of word c/32
-    auto scales_of = [&](int kb, float (&sc)[kT]) {
-      const uint32_t sw = load_scale_raw<FMT>(Ws, ws_row + kb);
+    // raw scale words of block kb: lane l holds the token scales l, l+32
+    // (0 for tokens >= M) and the weight scale; ring slot kb % kScaleAhead
+    uint32_t ra[kScaleAhead][kT], rw[kScaleAhead];
+    auto fetch = [&](int kb, uint32_t (&a)[kT], uint32_t& w) {
+      const bool in = kb < KB;
+      w = in ? load_scale_raw<FMT>(Ws, ws_row + kb) : 0u;
 #pragma unroll
       for (int t = 0; t < kT; ++t) {
         const int m = t * 32 + lane;
-        sc[t] = m < M ? combine_raw<FMT>(load_scale_raw<FMT>(Xs, static_cast<uint64_t>(kb) * ld_s + m), sw) : 0.0f;
+        a[t] = (in && m < M) ? load_scale_raw<FMT>(Xs, static_cast<uint64_t>(kb) * ld_s + m) : 0u;
       }
     };
+#pragma unroll
+    for (int d = 0; d < kScaleAhead; ++d) fetch(d, ra[d], rw[d]);
 
     bool ok = true;
-    float sc_next[kT];
-    scales_of(0, sc_next);
-    for (int kb = 0; kb < KB; ++kb) {
-      const int b = kb % C::kNumBuf;
-      float sc[kT];
+    for (int kb0 = 0; kb0 < KB && ok; kb0 += kScaleAhead) {
 #pragma unroll
-      for (int t = 0; t < kT; ++t) sc[t] = sc_next[t];
-      if (kb + 1 < KB) scales_of(kb + 1, sc_next);
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[b], (kb / C::kNumBuf) & 1u))) {
-        if (lane == 0) record_status(kDevTimeoutEpilogue);
-        ok = false;
-        break;
+      for (int d = 0; d < kScaleAhead; ++d) {
+        const int kb = kb0 + d;
+        if (kb >= KB) break;
+        float sc[kT];
+#pragma unroll
+        for (int t = 0; t < kT; ++t) sc[t] = (t * 32 + lane < M) ? combine_raw<FMT>(ra[d][t], rw[d]) : 0.0f;
+        fetch(kb + kScaleAhead, ra[d], rw[d]);
+        const int b = kb % C::kNumBuf;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[b], (kb / C::kNumBuf) & 1u))) {
+          if (lane == 0) record_status(kDevTimeoutEpilogue);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t taddr = taddr0 + static_cast<uint32_t>(b * BNT);
+        uint32_t p[BNT];
+#pragma unroll
+        for (int c = 0; c < BNT / 16; ++c)
+          tmem_ld_32x32b_x16(taddr + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&p[c * 16]));
+        tmem_wait_ld();
+#pragma unroll
+        for (int mm = 0; mm < BNT; ++mm) {
+          const float a = __shfl_sync(0xFFFFFFFFu, sc[mm / 32], mm % 32);
+          acc[mm] = __fmaf_rn(__uint_as_float(p[mm]), a, acc[mm]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[b]);
       }
-      tc_fence_after();
-      const uint32_t taddr = taddr0 + static_cast<uint32_t>(b * BNT);
-      uint32_t p[BNT];
-#pragma unroll
-      for (int c = 0; c < BNT / 16; ++c) tmem_ld_32x32b_x16(taddr + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&p[c * 16]));
-      tmem_wait_ld();
-#pragma unroll
-      for (int m = 0; m < BNT; ++m) {
-        const float a = __shfl_sync(0xFFFFFFFFu, sc[m / 32], m % 32);
-        acc[m] = __fmaf_rn(__uint_as_float(p[m]), a, acc[m]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[b]);
     }
     if (ok && n < N) {
 #pragma unroll
