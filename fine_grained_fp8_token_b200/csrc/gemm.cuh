@@ -57,10 +57,10 @@ struct GemmCfg {
   static constexpr size_t kSmemBytes = 1024 + kStages * static_cast<size_t>(kStageBytes) + kBarrierBytes;
   // 128 accumulators per thread need more than the launch share of
   // registers: warpgroup 0 gives some back (setmaxnreg) to the promotion
-  // warpgroups.  launch: 384 threads x 168 = 64512; after: 128 x 32 + 256 x 232.
+  // warpgroups.  launch: 384 threads x 168 = 64512; after: 128 x 24 + 256 x 240.
   static constexpr bool kRegSplit = CW > 64;
-  static constexpr int kRegsLow = 32;
-  static constexpr int kRegsHigh = 232;
+  static constexpr int kRegsLow = 24;
+  static constexpr int kRegsHigh = 240;
 };
 
 template <int N>
