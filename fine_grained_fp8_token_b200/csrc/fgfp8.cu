@@ -148,6 +148,18 @@ fgfp8_status launch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const 
   auto kernel = fgfp8::gemm_blockscaled_kernel<BN, CW, FMT, kGrouped>;
   st = set_smem(reinterpret_cast<const void*>(kernel), C::kSmemBytes, dev);
   if (st != FGFP8_OK) return st;
+  if (C::kRegSplit) {
+    // setmaxnreg.inc waits until registers are free: the warpgroups' shares
+    // must fit in what the block is launched with, or it would wait forever.
+    cudaFuncAttributes fa{};
+    cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
+    const long launch = static_cast<long>(fa.numRegs) * C::kThreads;
+    const long after = 128L * C::kRegsLow + static_cast<long>(C::kThreads - 128) * C::kRegsHigh;
+    if (after > launch)
+      return fail(FGFP8_ERR_UNSUPPORTED, "register split exceeds the launch allocation (" + std::to_string(fa.numRegs) +
+                                            " registers x " + std::to_string(C::kThreads) + " threads)");
+  }
   const int64_t tiles = ((M + C::kBM - 1) / C::kBM) * (N / BN);
   if (tiles == 0) return ok();
   const int64_t grid = tiles < sm_count ? tiles : sm_count;
@@ -157,29 +169,23 @@ fgfp8_status launch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const 
   return check_launch("gemm launch");
 }
 
-// Fraction of the last wave's CTA slots that hold work, for `tiles` tiles
-// spread over `sms` persistent CTAs.
-double wave_efficiency(int64_t tiles, int sms) {
-  const int64_t waves = (tiles + sms - 1) / sms;
-  return waves ? static_cast<double>(tiles) / static_cast<double>(waves * sms) : 1.0;
-}
-
 template <bool kGrouped>
 fgfp8_status dispatch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws, void* Y,
                            int64_t M, int64_t N, int64_t K, int fmt, const int32_t* offs, int E, int64_t b_rows,
                            cudaStream_t s, int dev, int sms) {
-  // 128x256 tiles halve the B traffic per MMA FLOP; 128x128 tiles when N is
-  // not a multiple of 256 or when they fill the last wave noticeably better.
-  const int64_t mt = (M + 127) / 128;
-  bool wide = (N % 256 == 0) && wave_efficiency(mt * (N / 256), sms) + 0.03 >= wave_efficiency(mt * (N / 128), sms);
+  // 128x256 tiles: measured faster per FLOP than 128x128 on B200 even where
+  // 128x128 tiles would fill the last wave better (4096^3: 95 us vs 119 us);
+  // 128x128 only when N is not a multiple of 256.
+  bool wide = (N % 256 == 0);
 #if defined(FGFP8_FORCE_BN)
   wide = (FGFP8_FORCE_BN == 256) && (N % 256 == 0);
 #endif
+  constexpr int kWideCW = 128;
   if (fmt == FGFP8_SCALE_F32) {
-    return wide ? launch_gemm<256, 128, 0, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms)
+    return wide ? launch_gemm<256, kWideCW, 0, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms)
                 : launch_gemm<128, 64, 0, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms);
   }
-  return wide ? launch_gemm<256, 128, 1, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms)
+  return wide ? launch_gemm<256, kWideCW, 1, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms)
               : launch_gemm<128, 64, 1, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms);
 }
 

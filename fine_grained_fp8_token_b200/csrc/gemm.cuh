@@ -55,12 +55,19 @@ struct GemmCfg {
   static constexpr int kStages = (224 * 1024) / kStageBytes;       // 7 (BN=128) or 4 (BN=256)
   static constexpr size_t kBarrierBytes = 256;
   static constexpr size_t kSmemBytes = 1024 + kStages * static_cast<size_t>(kStageBytes) + kBarrierBytes;
-  // 128 accumulators per thread need more than the launch share of
-  // registers: warpgroup 0 gives some back (setmaxnreg) to the promotion
-  // warpgroups.  launch: 384 threads x 168 = 64512; after: 128 x 24 + 256 x 240.
-  static constexpr bool kRegSplit = CW > 64;
+  // The promotion warps need more than an even share of the register file
+  // (CW fp32 accumulators per thread): warpgroup 0 gives registers back
+  // (setmaxnreg.dec) to the promotion warpgroups (setmaxnreg.inc).  The
+  // shares must sum to no more than the launch allocation (threads x the
+  // kernel's register count); the host checks the compiled count before the
+  // first launch.  384 threads x 168 = 128 x 24 + 256 x 240;
+  // 640 threads x 96 >= 128 x 24 + 512 x 112.
+  static constexpr int kLaunchRegs = (65536 / kThreads) & ~7;
+  static constexpr bool kRegSplit = true;
   static constexpr int kRegsLow = 24;
-  static constexpr int kRegsHigh = 240;
+  static constexpr int kRegsHigh = ((kThreads * kLaunchRegs - 128 * kRegsLow) / (kThreads - 128)) & ~7;
+  // columns loaded per tcgen05.wait::ld in the promotion loop
+  static constexpr int kPerWait = (CW >= 128) ? 64 : 16;
 };
 
 template <int N>
@@ -360,16 +367,18 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
           tc_fence_after();
           const uint32_t taddr = lane_base + static_cast<uint32_t>(buf * BN);
 #pragma unroll
-          for (int h = 0; h < CW / 64; ++h) {
-            uint32_t p0[32], p1[32];
-            tmem_ld_32x32b_x32(taddr + h * 64, p0);
-            tmem_ld_32x32b_x32(taddr + h * 64 + 32, p1);
+          for (int h = 0; h < CW / C::kPerWait; ++h) {
+            uint32_t p[C::kPerWait];
+            if (C::kPerWait == 64) {
+              tmem_ld_32x32b_x32(taddr + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&p[0]));
+              tmem_ld_32x32b_x32(taddr + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&p[C::kPerWait / 2]));
+            } else {
+              tmem_ld_32x32b_x16(taddr + h * 16, *reinterpret_cast<uint32_t(*)[16]>(&p[0]));
+            }
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) acc[h * 64 + j] = __fmaf_rn(__uint_as_float(p0[j]), sc, acc[h * 64 + j]);
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              acc[h * 64 + 32 + j] = __fmaf_rn(__uint_as_float(p1[j]), sc, acc[h * 64 + 32 + j]);
+            for (int j = 0; j < C::kPerWait; ++j)
+              acc[h * C::kPerWait + j] = __fmaf_rn(__uint_as_float(p[j]), sc, acc[h * C::kPerWait + j]);
           }
           tc_fence_before();
           __syncwarp();
