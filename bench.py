@@ -66,6 +66,32 @@ def measured_peaks():
     return {**FALLBACK_PEAKS, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def kernel_source_sha256():
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "fine_grained_fp8_token_b200", "csrc", "*"))):
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def ncu_traffic(workload_name):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, or None when there is none for this workload or the kernel
+    sources changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            cap = json.load(f)["captures"].get(workload_name)
+    except (OSError, ValueError, KeyError):
+        return None
+    if not cap or cap.get("source_sha256") != kernel_source_sha256():
+        return None
+    return cap["dram_read_bytes"] + cap["dram_write_bytes"]
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     """SM clock and throttle reasons of this GPU, sampled every 10 ms through
@@ -193,6 +219,9 @@ class DenseLayer:
     def host_io(self):
         return self.X, self.Y
 
+    def gemm_kernel_name(self):
+        return "gemm_decode_kernel" if self.cfg.M <= 64 else "gemm_blockscaled_kernel"
+
 
 class MoELayer:
     """Grouped expert layer: routed token rows and pre-quantized experts."""
@@ -251,6 +280,9 @@ class MoELayer:
 
     def host_io(self):
         return self.X, self.Y
+
+    def gemm_kernel_name(self):
+        return "gemm_blockscaled_kernel (grouped)"
 
 
 def make_layer(name, dev):
@@ -484,12 +516,13 @@ def main():
     hbm_bound = gemm_tflops / fp8_peak < gemm_gbs / peaks["hbm_gbs"]
     if hbm_bound:
         roofline = {"bound": "hbm", "achieved": gemm_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": gemm_gbs / peaks["hbm_gbs"], "traffic": None,
-                    "kernel": "gemm_blockscaled_kernel",
+                    "frac": gemm_gbs / peaks["hbm_gbs"], "traffic": ncu_traffic(layer.describe()["workload"]),
+                    "kernel": layer.gemm_kernel_name(),
                     "peak_source": f"{peaks['source']} HBM copy bandwidth"}
     else:
         roofline = {"bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
-                    "frac": gemm_tflops / fp8_peak, "traffic": None, "kernel": "gemm_blockscaled_kernel",
+                    "frac": gemm_tflops / fp8_peak, "traffic": ncu_traffic(layer.describe()["workload"]),
+                    "kernel": layer.gemm_kernel_name(),
                     "peak_source": f"{peaks['source']} cuBLAS bf16 burst x {FP8_OVER_BF16:g} (nominal fp8/bf16)"}
     line = {
         "impl": "fgfp8", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": n,
