@@ -51,7 +51,7 @@ WORKLOAD_ALIASES = {
     "llama_attn": workloads.LLAMA_ATTN.name, "tiny": workloads.TINY.name,
     "llama_gate_up": workloads.LLAMA_GATE_UP.name, "llama_down": workloads.LLAMA_DOWN.name,
     **{f"ds_decode_m{m}": workloads.DS_DECODE[m].name for m in (1, 8, 32, 64)},
-    "moe": workloads.MOE.name,
+    "moe": workloads.MOE.name, "moe_small": workloads.MOE_SMALL.name,
 }
 
 
@@ -287,8 +287,9 @@ class MoELayer:
 
 def make_layer(name, dev):
     name = WORKLOAD_ALIASES.get(name, name)
-    if name == workloads.MOE.name:
-        return MoELayer(workloads.MOE, dev)
+    for cfg in (workloads.MOE, workloads.MOE_SMALL):
+        if name == cfg.name:
+            return MoELayer(cfg, dev)
     return DenseLayer(workloads.LINEARS[name], dev)
 
 
@@ -394,8 +395,8 @@ class OracleSample:
         import oracle
         self.oracle = oracle
         name = WORKLOAD_ALIASES.get(name, name)
-        if name == workloads.MOE.name:
-            cfg = workloads.MOE
+        if name in (workloads.MOE.name, workloads.MOE_SMALL.name):
+            cfg = workloads.MOE if name == workloads.MOE.name else workloads.MOE_SMALL
             r = workloads.moe_routing(cfg)
             e = int(np.argmax(r.counts))                    # the busiest expert's rows
             tok = r.row_token[r.group_offs[e]:r.group_offs[e] + r.counts[e]]

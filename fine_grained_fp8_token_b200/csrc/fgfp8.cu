@@ -169,6 +169,32 @@ fgfp8_status launch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const 
   return check_launch("gemm launch");
 }
 
+// UE8M0 launch with hardware block scaling (persistent, 128 x BN tiles).
+template <int BN, bool kGrouped>
+fgfp8_status launch_gemm_mx(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
+                            void* Y, int64_t M, int64_t N, int64_t K, const int32_t* offs, int E, int64_t b_rows,
+                            cudaStream_t stream, int dev, int sm_count) {
+  using C = fgfp8::MxCfg<BN>;
+  CUtensorMap mA, mB;
+  fgfp8_status st = make_map_u8_sw128(&mA, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
+                                      static_cast<uint64_t>(K), 128);
+  if (st != FGFP8_OK) return st;
+  st = make_map_u8_sw128(&mB, Wq, static_cast<uint64_t>(b_rows), static_cast<uint64_t>(K), static_cast<uint64_t>(K),
+                         C::kBN);
+  if (st != FGFP8_OK) return st;
+  auto kernel = fgfp8::gemm_mx_kernel<BN, kGrouped>;
+  st = set_smem(reinterpret_cast<const void*>(kernel), C::kSmemBytes, dev);
+  if (st != FGFP8_OK) return st;
+  const int64_t tiles = ((M + C::kBM - 1) / C::kBM) * (N / C::kBN);
+  if (tiles == 0) return ok();
+  const int64_t grid = tiles < sm_count ? tiles : sm_count;
+  kernel<<<static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, stream>>>(
+      mA, mB, reinterpret_cast<const uint8_t*>(Xs), static_cast<uint32_t>(ld_s), reinterpret_cast<const uint8_t*>(Ws),
+      reinterpret_cast<__nv_bfloat16*>(Y), static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), offs, E,
+      static_cast<int>(tiles));
+  return check_launch("block-scaled gemm launch");
+}
+
 template <bool kGrouped>
 fgfp8_status dispatch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws, void* Y,
                            int64_t M, int64_t N, int64_t K, int fmt, const int32_t* offs, int E, int64_t b_rows,
@@ -181,12 +207,12 @@ fgfp8_status dispatch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, cons
   wide = (FGFP8_FORCE_BN == 256) && (N % 256 == 0);
 #endif
   constexpr int kWideCW = 128;
-  if (fmt == FGFP8_SCALE_F32) {
-    return wide ? launch_gemm<256, kWideCW, 0, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms)
-                : launch_gemm<128, 64, 0, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms);
-  }
-  return wide ? launch_gemm<256, kWideCW, 1, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms)
-              : launch_gemm<128, 64, 1, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms);
+  // UE8M0 scales: the tensor core applies them (block-scaled MMA), no promotion.
+  if (fmt == FGFP8_SCALE_UE8M0)
+    return wide ? launch_gemm_mx<256, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms)
+                : launch_gemm_mx<128, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms);
+  return wide ? launch_gemm<256, kWideCW, 0, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms)
+              : launch_gemm<128, 64, 0, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms);
 }
 
 // Few-token (M <= 64) launch: one CTA per 128 output columns, operands swapped.

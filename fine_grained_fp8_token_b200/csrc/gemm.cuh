@@ -155,6 +155,7 @@ __device__ __forceinline__ void issue_mmas(uint32_t a_base, uint32_t b_base, int
                                            uint64_t* full, uint64_t* empty, uint64_t* tfull, uint64_t* tempty,
                                            uint64_t* mma_done) {
   constexpr uint32_t idesc = idesc_e4m3_f32(128, kN);
+  const uint64_t a_desc0 = smem_desc_k_sw128(a_base), b_desc0 = smem_desc_k_sw128(b_base);
   for (int kb = 0; kb < KB; ++kb) {
     const int s = kb % kStages;
     const int b = kb % kNumBuf;
@@ -170,8 +171,8 @@ __device__ __forceinline__ void issue_mmas(uint32_t a_base, uint32_t b_base, int
     const uint32_t d = tmem_base + static_cast<uint32_t>(b * kN);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
-      const uint64_t ad = smem_desc_k_sw128(a_base + s * kABytes + kk * 32);
-      const uint64_t bd = smem_desc_k_sw128(b_base + s * kBBytes + kk * 32);
+      const uint64_t ad = a_desc0 + ((s * kABytes + kk * 32) >> 4);
+      const uint64_t bd = b_desc0 + ((s * kBBytes + kk * 32) >> 4);
       mma_f8f6f4(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
     }
     mma_commit(&empty[s]);
@@ -281,6 +282,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
       // ================= MMA issuer
       constexpr uint32_t idesc = idesc_e4m3_f32(128, BN);
       const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
+      // descriptors differ per stage / K step only in the start-address field
+      const uint64_t a_desc0 = smem_desc_k_sw128(a_base), b_desc0 = smem_desc_k_sw128(b_base);
       uint32_t it = 0, bt = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
@@ -305,8 +308,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
           const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = smem_desc_k_sw128(a_base + s * C::kABytes + kk * 32);
-            const uint64_t bd = smem_desc_k_sw128(b_base + s * C::kBBytes + kk * 32);
+            const uint64_t ad = a_desc0 + ((s * C::kABytes + kk * 32) >> 4);
+            const uint64_t bd = b_desc0 + ((s * C::kBBytes + kk * 32) >> 4);
             mma_f8f6f4(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
           }
           mma_commit(&empty[s]);
@@ -406,6 +409,287 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
   }
 
   // ---- teardown
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+// ---------------------------------------------------------------------------
+// UE8M0 variant with hardware block scaling ("UE8M0 scale format": scales are
+// powers of two, which the tensor core can apply itself).  Per 128-wide K
+// block the MMA takes one UE8M0 scale per row of Xq and one per row of Wq
+// (the 128x128 weight block's scale, shared by its 128 rows) from TMEM
+// (kind::mxf8f6f4.block_scale, one scale per 32-element K slice; the four
+// slices of a 128 block use the same scale), so the whole K reduction
+// accumulates in TMEM and no promotion step runs per K block.
+//   warp 0      TMA for the operand tiles (lane 0) and, with all 32 lanes,
+//               the scale rows of each K block written to shared memory in
+//               the TMEM scale layout (lane l: scales of rows l, l+32, l+64,
+//               l+96, each byte repeated for the four K slices);
+//   warp 1      owns TMEM: per K block tcgen05.cp of the two scale tiles
+//               into TMEM, then four block-scaled MMAs; after the tile's last
+//               K block it publishes the accumulator (two buffers, so the
+//               epilogue of one tile overlaps the MMAs of the next);
+//   warps 4..7  epilogue: TMEM -> registers -> bf16 -> global.
+// TMEM: accumulators in columns [0, 256) (2 x 128), scale factors in
+// [256, 272) (2 K-block parities x (4 columns for A + 4 for B)).
+// ---------------------------------------------------------------------------
+template <int BN>
+struct MxCfg {
+  static constexpr int kBM = 128, kBN = BN, kBK = 128;
+  static constexpr int kEpiWarps = 4 * (BN / 128);                 // one warp per 32 rows x 128 columns
+  static constexpr int kThreads = 128 + 32 * kEpiWarps;
+  static constexpr int kNumAcc = (BN == 128) ? 2 : 1;             // accumulator buffers in TMEM
+  static constexpr uint32_t kABytes = kBM * kBK;
+  static constexpr uint32_t kBBytes = kBN * kBK;
+  static constexpr uint32_t kSfABytes = 512;                      // 32 rows x 16 bytes (128 rows of A)
+  static constexpr uint32_t kSfBBytes = 512 * (BN / 128);         // one 32 x 16 tile per 128 rows of B
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes;      // TMA bytes per stage
+  static constexpr int kStages = (BN == 128) ? 6 : 4;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kSfCol = kNumAcc * BN;                // scale factors after the accumulators
+  static constexpr uint32_t kSfColsPerKb = 4 + BN / 32;           // A: 4 columns, B: BN/32 columns
+  static constexpr size_t kBarrierBytes = 256;
+  static constexpr size_t kSmemBytes =
+      1024 + kStages * static_cast<size_t>(kStageBytes + kSfABytes + kSfBBytes) + kBarrierBytes;
+  static constexpr int kPrefetch = 4;                             // scale prefetch depth (K blocks)
+};
+
+template <int BN, bool kGrouped>
+__global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
+    gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const uint8_t* __restrict__ Xs, uint32_t ld_s, const uint8_t* __restrict__ Ws,
+                   __nv_bfloat16* __restrict__ Y, int M, int N, int K, const int32_t* __restrict__ group_offs,
+                   int E, int num_tiles) {
+  using C = MxCfg<BN>;
+  static_assert(C::kSfCol + 2 * C::kSfColsPerKb <= C::kTmemCols, "TMEM columns");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + C::kStages * C::kABytes;
+  uint8_t* sSfA = sB + C::kStages * C::kBBytes;
+  uint8_t* sSfB = sSfA + C::kStages * C::kSfABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sSfB + C::kStages * C::kSfBBytes);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* mma_done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int KB = K / C::kBK;
+  const int NB = N / 128;
+  const int num_m = (M + C::kBM - 1) / C::kBM;
+  const int num_n = N / C::kBN;
+
+  auto coords = [&](int t, int& m0, int& n0, int& expert) {
+    if (!kGrouped) {
+      m0 = (t % num_m) * C::kBM;
+      n0 = (t / num_m) * C::kBN;
+      expert = 0;
+    } else {
+      n0 = (t % num_n) * C::kBN;
+      m0 = (t / num_n) * C::kBM;
+      expert = find_expert(group_offs, E, m0);
+    }
+  };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 2);                  // TMA bytes (+1 arrival) and the scale rows (+1 arrival)
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], C::kEpiWarps);
+    }
+    mbar_init(mma_done, 1);
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ================= producer: TMA (lane 0) + scale rows (all lanes)
+    uint32_t it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      int m0, n0, expert;
+      coords(t, m0, n0, expert);
+      if (expert < 0) {
+        if (lane == 0) record_status(kDevBadGroupOffsets);
+        continue;
+      }
+      const uint64_t ws_row = (static_cast<uint64_t>(expert) * NB + n0 / 128) * KB;
+      // prefetched scale bytes: rows lane + 32 j of the tile's A rows, and the
+      // scale of each 128-row weight block of the tile
+      uint32_t pa[C::kPrefetch][4], pw[C::kPrefetch][BN / 128];
+      auto fetch = [&](int kb, uint32_t (&a)[4], uint32_t (&w)[BN / 128]) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int m = m0 + lane + 32 * j;
+          a[j] = (kb < KB && m < M) ? __ldg(Xs + static_cast<uint64_t>(kb) * ld_s + m) : 127u;
+        }
+#pragma unroll
+        for (int h = 0; h < BN / 128; ++h) w[h] = kb < KB ? __ldg(Ws + ws_row + static_cast<uint64_t>(h) * KB + kb) : 127u;
+      };
+#pragma unroll
+      for (int d = 0; d < C::kPrefetch; ++d) fetch(d, pa[d], pw[d]);
+      for (int kb0 = 0; kb0 < KB && ok; kb0 += C::kPrefetch) {
+#pragma unroll
+        for (int d = 0; d < C::kPrefetch; ++d) {
+          const int kb = kb0 + d;
+          if (kb >= KB) break;
+          const int s = it % C::kStages;
+          if (!__all_sync(0xFFFFFFFFu, it < static_cast<uint32_t>(C::kStages) ||
+                                           mbar_wait(&empty[s], ((it / C::kStages) & 1u) ^ 1u))) {
+            if (lane == 0) record_status(kDevTimeoutProducer);
+            ok = false;
+            break;
+          }
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+            tma_load_2d(sA + s * C::kABytes, &tmA, &full[s], kb * C::kBK, m0);
+            tma_load_2d(sB + s * C::kBBytes, &tmB, &full[s], kb * C::kBK, expert * N + n0);
+          }
+          // scale rows in the TMEM scale layout: lane l holds rows l + 32 j,
+          // each byte repeated for the four 32-element K slices
+          uint4 ra;
+          ra.x = pa[d][0] * 0x01010101u;
+          ra.y = pa[d][1] * 0x01010101u;
+          ra.z = pa[d][2] * 0x01010101u;
+          ra.w = pa[d][3] * 0x01010101u;
+          *reinterpret_cast<uint4*>(sSfA + s * C::kSfABytes + lane * 16) = ra;
+#pragma unroll
+          for (int h = 0; h < BN / 128; ++h) {
+            const uint32_t w4 = pw[d][h] * 0x01010101u;
+            *reinterpret_cast<uint4*>(sSfB + s * C::kSfBBytes + h * 512 + lane * 16) = make_uint4(w4, w4, w4, w4);
+          }
+          fetch(kb + C::kPrefetch, pa[d], pw[d]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full[s]);
+          ++it;
+        }
+      }
+    }
+    if (lane == 0) {
+      for (uint32_t j = (it > static_cast<uint32_t>(C::kStages) ? it - C::kStages : 0); j < it; ++j)
+        if (!mbar_wait(&full[j % C::kStages], (j / C::kStages) & 1u)) record_status(kDevTimeoutProducer);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ================= MMA issuer
+      constexpr uint32_t idesc = idesc_mx_e4m3_ue8m0(128, C::kBN);
+      const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
+      // descriptors differ per stage / K step only in the start-address field
+      const uint64_t a_desc0 = smem_desc_k_sw128(a_base), b_desc0 = smem_desc_k_sw128(b_base);
+      const uint64_t sfa_desc0 = smem_desc_rows16(smem_u32(sSfA)), sfb_desc0 = smem_desc_rows16(smem_u32(sSfB));
+      uint32_t it = 0, tile_no = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        int m0, n0, expert;
+        coords(t, m0, n0, expert);
+        if (expert < 0) continue;
+        const int ab = tile_no % C::kNumAcc;            // accumulator buffer
+        const int tb = tile_no & 1;                      // tfull / tempty barrier of this tile
+        if (tile_no >= static_cast<uint32_t>(C::kNumAcc) &&
+            !mbar_wait(&tempty[(tile_no - C::kNumAcc) & 1], ((tile_no - C::kNumAcc) >> 1) & 1u)) {
+          record_status(kDevTimeoutMma);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(ab * C::kBN);
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % C::kStages;
+          if (!mbar_wait(&full[s], (it / C::kStages) & 1u)) {
+            record_status(kDevTimeoutMma);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sfa = tmem_base + C::kSfCol + static_cast<uint32_t>((kb & 1) * C::kSfColsPerKb);
+          const uint32_t sfb = sfa + 4;
+          tmem_cp_32x128b_x4(sfa, sfa_desc0 + ((s * C::kSfABytes) >> 4));
+#pragma unroll
+          for (int h = 0; h < BN / 128; ++h)
+            tmem_cp_32x128b_x4(sfb + 4 * h, sfb_desc0 + ((s * C::kSfBBytes + h * 512) >> 4));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t adesc = a_desc0 + ((s * C::kABytes + kk * 32) >> 4);
+            const uint64_t bdesc = b_desc0 + ((s * C::kBBytes + kk * 32) >> 4);
+            mma_mxf8f6f4(d, adesc, bdesc, idesc, sfa, sfb, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&empty[s]);
+        }
+        if (ok) mma_commit(&tfull[tb]);
+        ++tile_no;
+      }
+      mma_commit(mma_done);
+      if (!mbar_wait(mma_done, 0)) record_status(kDevTimeoutMma);
+    }
+  } else if (warp >= 4) {
+    // ================= epilogue: TMEM -> bf16 -> global
+    const int ew = warp - 4;
+    const int quad = warp & 3;
+    const int col0 = (ew >> 2) * 128;
+    const int row = quad * 32 + lane;
+    uint32_t tile_no = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      int m0, n0, expert;
+      coords(t, m0, n0, expert);
+      if (expert < 0) continue;
+      const int ab = tile_no % C::kNumAcc;
+      const int tb = tile_no & 1;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[tb], (tile_no >> 1) & 1u))) {
+        if (lane == 0) record_status(kDevTimeoutEpilogue);
+        break;
+      }
+      tc_fence_after();
+      const int m = m0 + row;
+      const uint32_t taddr =
+          tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(ab * C::kBN + col0);
+      __nv_bfloat16* yrow = Y + static_cast<uint64_t>(m) * N + n0 + col0;
+#pragma unroll
+      for (int h = 0; h < 128 / 32; ++h) {
+        uint32_t p[32];
+        tmem_ld_32x32b_x32(taddr + h * 32, p);
+        tmem_wait_ld();
+        if (m < M) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            uint4 v;
+            __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(p[j + 0]), __uint_as_float(p[j + 1]));
+            __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(p[j + 2]), __uint_as_float(p[j + 3]));
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(p[j + 4]), __uint_as_float(p[j + 5]));
+            __nv_bfloat162 h3 = __floats2bfloat162_rn(__uint_as_float(p[j + 6]), __uint_as_float(p[j + 7]));
+            v.x = *reinterpret_cast<uint32_t*>(&h0);
+            v.y = *reinterpret_cast<uint32_t*>(&h1);
+            v.z = *reinterpret_cast<uint32_t*>(&h2);
+            v.w = *reinterpret_cast<uint32_t*>(&h3);
+            *reinterpret_cast<uint4*>(yrow + h * 32 + j) = v;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[tb]);
+      ++tile_no;
+    }
+  }
+
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

@@ -179,6 +179,33 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
       : "r"(taddr));
 }
 
+// ------------------------------------------------------------ block-scaled MMA (UE8M0)
+// D[tmem] (+)= (A * 2^(sfa-127)) x (B * 2^(sfb-127))^T with one UE8M0 scale
+// per row and 32-element K slice (kind::mxf8f6f4.block_scale, scale_vec 1X),
+// scales read from TMEM at sfa / sfb.
+__device__ __forceinline__ void mma_mxf8f6f4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t tmem_sfa, uint32_t tmem_sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(tmem_sfa), "r"(tmem_sfb), "r"(accumulate)
+      : "memory");
+}
+
+// Copy a 32-row x 16-byte shared-memory tile (no swizzle, rows 16 bytes
+// apart) into TMEM columns [taddr, taddr+4) of lanes 0-31, replicated into
+// all four 32-lane subpartitions (32x128b.warpx4).
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Make this thread's generic-proxy shared-memory writes visible to the async
+// proxy (TMA, tcgen05.cp, tcgen05.mma operand reads).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ------------------------------------------------------------ UMMA descriptors
 // Shared-memory matrix descriptor for a K-major operand tile written by TMA
 // with 128-byte swizzling: rows of 128 bytes, 8-row core groups 1024 bytes
@@ -194,6 +221,26 @@ __device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t smem_addr) {
   d |= static_cast<uint64_t>(1u) << 46;
   d |= static_cast<uint64_t>(2u) << 61;
   return d;
+}
+
+// Shared-memory descriptor for an unswizzled K-major tile whose rows are 16
+// bytes apart (core matrices of 8 rows x 16 bytes, 128 bytes apart): the
+// source layout of tcgen05.cp 32x128b.
+__device__ __forceinline__ uint64_t smem_desc_rows16(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(128u >> 4) << 16;        // leading byte offset (one 16-byte chunk per row)
+  d |= static_cast<uint64_t>(128u >> 4) << 32;        // stride byte offset: 8-row groups 128 bytes apart
+  d |= static_cast<uint64_t>(1u) << 46;               // descriptor version
+  return d;                                            // layout 0: no swizzle
+}
+
+// Instruction descriptor, kind::mxf8f6f4.block_scale: E4M3 x E4M3, fp32
+// accumulate, both K-major, UE8M0 scales (bit 23), scale-factor byte ids 0,
+// K = 32 (bit 31 clear).  b_sf_id bits 4-5, a/b formats 7-9 / 10-12, N>>3 at
+// 17-22, M>>4 at 24-28, a_sf_id 29-30.
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3_ue8m0(int M, int N) {
+  return (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 // Instruction descriptor, kind::f8f6f4: E4M3 x E4M3 -> F32, both K-major,

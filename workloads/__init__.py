@@ -63,6 +63,9 @@ LLAMA_DOWN = Linear("llama3_8b_down_8192x4096x14336", 8192, 4096, 14336, SCALE_F
 DS_DECODE = {m: Linear(f"deepseek_v3_decode_m{m}_18432x7168", m, 18432, 7168, SCALE_UE8M0,
                        x_kind="normal") for m in (1, 8, 32, 64)}
 MOE = MoE("deepseek_v3_moe_256x4096x7168_top8")
+# the same expert shapes with 32 experts and 512 tokens (~1 GB of weights): a
+# profiling case larger than L2 but small enough for multi-pass captures
+MOE_SMALL = MoE("deepseek_v3_moe_32x4096x7168_top8_512tok", E=32, tokens=512)
 
 LINEARS = {c.name: c for c in [TINY, LLAMA_ATTN, LLAMA_GATE_UP, LLAMA_DOWN, *DS_DECODE.values()]}
 
