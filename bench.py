@@ -293,6 +293,24 @@ def make_layer(name, dev):
     return DenseLayer(workloads.LINEARS[name], dev)
 
 
+# ---------------------------------------------------------------- ranks
+def max_over_ranks(times, world, device):
+    """Element-wise max of per-rank timings: the job takes as long as its
+    slowest replica.  Every rank calls this exactly once per run, in the same
+    order, so the collective sequence matches on all ranks."""
+    t = torch.tensor([float(x) for x in times], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_rate(world, units_per_rank, ms):
+    """Units processed by all ranks per second, in units / 1e12 (TFLOP/s for
+    FLOPs), when each of `world` replicas processes `units_per_rank` and the
+    slowest takes `ms` milliseconds."""
+    return world * units_per_rank / (ms / 1e3) / 1e12
+
+
 # ---------------------------------------------------------------- timing
 def run_gpu(args, rank, world, dev):
     layer = make_layer(args.workload, dev)
@@ -369,11 +387,9 @@ def run_gpu(args, rank, world, dev):
     h2d = X_host.numel() * X_host.element_size()
     d2h = Y_host.numel() * Y_host.element_size()
 
-    stats = torch.tensor([total_ms, sum(gemm_ms), sum(quant_ms), statistics.mean(e2e_ms),
-                          statistics.mean(wq_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(stats, op=torch.distributed.ReduceOp.MAX)
-    total_ms, gemm_total, quant_total, e2e_mean, wq_mean = stats.tolist()
+    total_ms, gemm_total, quant_total, e2e_mean, wq_mean = max_over_ranks(
+        [total_ms, sum(gemm_ms), sum(quant_ms), statistics.mean(e2e_ms), statistics.mean(wq_ms)],
+        world, dev)
     return layer, {"total_ms": total_ms, "gemm_ms": gemm_total / n, "quant_ms": quant_total / n,
                    "e2e_ms": e2e_mean, "wq_ms": wq_mean, "clocks": clocks, "h2d": h2d, "d2h": d2h,
                    "launches": launches_per_step * n}
@@ -447,12 +463,21 @@ def cpu_baseline(name, target_s=15.0):
                       f"{reps} steps of {dt:.2f} s"}
 
 
+REFERENCE_RUN_SECONDS = 150.0
+
+
+def reference_step_seconds(steps, warmup, budget_s=REFERENCE_RUN_SECONDS):
+    """Target duration of one oracle step so that warm-up plus timed steps end
+    within about budget_s (at most 2 s a step)."""
+    return min(2.0, budget_s / max(1, steps + warmup))
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     os.environ.setdefault("OMP_NUM_THREADS", str(cpu_cores()))
-    s = calibrated_sample(args.workload, 2.0)
+    s = calibrated_sample(args.workload, reference_step_seconds(args.steps, args.warmup))
     for _ in range(args.warmup):
         s.step()
     times = []
@@ -508,7 +533,7 @@ def main():
     n = args.steps
     step_ms = r["total_ms"] / n
     flops = layer.flops()
-    value = world * flops / (step_ms / 1e3) / 1e12
+    value = whole_job_rate(world, flops, step_ms)
     fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
     gemm_tflops = flops / (r["gemm_ms"] / 1e3) / 1e12
     gemm_gbs = layer.gemm_bytes() / (r["gemm_ms"] / 1e3) / 1e9
@@ -540,7 +565,7 @@ def main():
             "quant_weight_offline": {"us": 1e3 * r["wq_ms"], "gbs": wq_gbs, "frac_hbm": wq_gbs / peaks["hbm_gbs"],
                                      "bytes": layer.weight_bytes()},
         },
-        "e2e": {"value": world * flops / (r["e2e_ms"] / 1e3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": whole_job_rate(world, flops, r["e2e_ms"]), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"], "ms_per_step": r["e2e_ms"]},
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
