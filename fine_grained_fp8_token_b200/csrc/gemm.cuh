@@ -52,9 +52,14 @@ struct GemmCfg {
   static constexpr uint32_t kABytes = kBM * kBK;
   static constexpr uint32_t kBBytes = BN * kBK;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = (224 * 1024) / kStageBytes;       // 7 (BN=128) or 4 (BN=256)
+  // Epilogue staging: each promotion warp transposes its 32 rows x 64
+  // columns of bf16 (4 KB) per pass through its own slot.
+  static constexpr uint32_t kWarpStageBytes = 32 * 128;
+  static constexpr uint32_t kStagingBytes = kEpiWarps * kWarpStageBytes;
+  static constexpr int kStages = (224 * 1024 - kStagingBytes) / kStageBytes;  // 6 (BN=128) or 4 (BN=256)
   static constexpr size_t kBarrierBytes = 256;
-  static constexpr size_t kSmemBytes = 1024 + kStages * static_cast<size_t>(kStageBytes) + kBarrierBytes;
+  static constexpr size_t kSmemBytes =
+      1024 + kStages * static_cast<size_t>(kStageBytes) + kStagingBytes + kBarrierBytes;
   // The promotion warps need more than an even share of the register file
   // (CW fp32 accumulators per thread): warpgroup 0 gives registers back
   // (setmaxnreg.dec) to the promotion warpgroups (setmaxnreg.inc).  The
@@ -193,7 +198,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::kStages * C::kABytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::kStages * C::kBBytes);
+  uint8_t* sStg = sB + C::kStages * C::kBBytes;       // epilogue staging, one slot per promotion warp
+  uint64_t* full = reinterpret_cast<uint64_t*>(sStg + C::kStagingBytes);
   uint64_t* empty = full + C::kStages;
   uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + C::kNumBuf;
@@ -324,31 +330,41 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
     // ================= promotion / epilogue
     const int ew = warp - 4;
     const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
-    const int col0 = (ew >> 2) * CW;
+    const int grp = ew >> 2;                   // column group: columns [grp * CW, grp * CW + CW)
+    const int col0 = grp * CW;
     const int row = quad * 32 + lane;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(col0);
+    // raw scale words for K blocks kb .. kb+kScaleAhead-1, ring slot kb % kScaleAhead
+    uint32_t ra[kScaleAhead], rw[kScaleAhead];
+    auto fetch = [&](int kb, int m, bool live, uint64_t ws_row, uint32_t& a, uint32_t& w) {
+      if (live && kb < KB) {
+        a = load_scale_raw<FMT>(Xs, static_cast<uint64_t>(kb) * ld_s + m);
+        w = load_scale_raw<FMT>(Ws, ws_row + kb);
+      } else {
+        a = 0u;
+        w = 0u;
+      }
+    };
+    // this thread's row, liveness and weight-scale row in tile t (expert < 0: skipped tile)
+    auto tile_rows = [&](int t, int& m0, int& n0, int& expert, int& m, bool& live, uint64_t& ws_row) {
+      coords(t, m0, n0, expert);
+      m = m0 + row;
+      live = (m < M) && (n0 + col0 < N);
+      ws_row = (static_cast<uint64_t>(expert < 0 ? 0 : expert) * NB + (n0 + col0) / 128) * KB;
+    };
+    int pref_t = -1;                           // tile whose first scale words are in the ring
     uint32_t bt = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-      int m0, n0, expert;
-      coords(t, m0, n0, expert);
+      int m0, n0, expert, m;
+      bool live;
+      uint64_t ws_row;
+      tile_rows(t, m0, n0, expert, m, live, ws_row);
       if (expert < 0) continue;
-      const int m = m0 + row;
-      const bool live = (m < M) && (n0 + col0 < N);
-      const uint64_t ws_row = (static_cast<uint64_t>(expert) * NB + (n0 + col0) / 128) * KB;
-      // raw scale words for K blocks kb .. kb+kScaleAhead-1, ring slot kb % kScaleAhead
-      uint32_t ra[kScaleAhead], rw[kScaleAhead];
-      auto fetch = [&](int kb, uint32_t& a, uint32_t& w) {
-        if (live && kb < KB) {
-          a = load_scale_raw<FMT>(Xs, static_cast<uint64_t>(kb) * ld_s + m);
-          w = load_scale_raw<FMT>(Ws, ws_row + kb);
-        } else {
-          a = 0u;
-          w = 0u;
-        }
-      };
+      if (pref_t != t) {
 #pragma unroll
-      for (int d = 0; d < kScaleAhead; ++d) fetch(d, ra[d], rw[d]);
+        for (int d = 0; d < kScaleAhead; ++d) fetch(d, m, live, ws_row, ra[d], rw[d]);
+      }
 
       float acc[CW];
 #pragma unroll
@@ -359,7 +375,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
           const int kb = kb0 + d;
           if (kb >= KB) break;
           const float sc = live ? combine_raw<FMT>(ra[d], rw[d]) : 0.0f;
-          fetch(kb + kScaleAhead, ra[d], rw[d]);
+          fetch(kb + kScaleAhead, m, live, ws_row, ra[d], rw[d]);
           const int buf = bt % C::kNumBuf;
           // warp-uniform outcome: the TMEM loads below are .sync.aligned
           if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[buf], (bt / C::kNumBuf) & 1u))) {
@@ -389,10 +405,34 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
           ++bt;
         }
       }
-      if (ok && live) {
-        __nv_bfloat16* yrow = Y + static_cast<uint64_t>(m) * N + n0 + col0;
+      if (!ok) break;
+
+      // The next tile's first scale words: their latency overlaps the epilogue.
+      pref_t = -1;
+      if (t + static_cast<int>(gridDim.x) < num_tiles) {
+        const int tn = t + static_cast<int>(gridDim.x);
+        int m0n, n0n, en, mn;
+        bool liven;
+        uint64_t wsn;
+        tile_rows(tn, m0n, n0n, en, mn, liven, wsn);
+        if (en >= 0) {
 #pragma unroll
-        for (int j = 0; j < CW; j += 8) {
+          for (int d = 0; d < kScaleAhead; ++d) fetch(d, mn, liven, wsn, ra[d], rw[d]);
+          pref_t = tn;
+        }
+      }
+
+      // Epilogue: bf16 (round-to-nearest-even), transposed through the warp's
+      // shared-memory slot so that each store instruction writes four whole
+      // 128-byte row segments.  Per 64-column pass, lane l writes its row's
+      // eight 16-byte chunks (chunk c at position c ^ (l % 8): conflict-free),
+      // then reads back row 4i + l / 8, chunk l % 8, for i = 0..7.
+      uint8_t* slot = sStg + ew * C::kWarpStageBytes;
+#pragma unroll
+      for (int p = 0; p < CW / 64; ++p) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const int j = p * 64 + c * 8;
           uint4 v;
           __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[j + 0], acc[j + 1]);
           __nv_bfloat162 h1 = __floats2bfloat162_rn(acc[j + 2], acc[j + 3]);
@@ -402,8 +442,17 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
           v.y = *reinterpret_cast<uint32_t*>(&h1);
           v.z = *reinterpret_cast<uint32_t*>(&h2);
           v.w = *reinterpret_cast<uint32_t*>(&h3);
-          *reinterpret_cast<uint4*>(yrow + j) = v;
+          *reinterpret_cast<uint4*>(slot + lane * 128 + ((c ^ (lane & 7)) << 4)) = v;
         }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = 4 * i + (lane >> 3), c = lane & 7;
+          const uint4 v = *reinterpret_cast<const uint4*>(slot + r * 128 + ((c ^ (r & 7)) << 4));
+          const int mr = m0 + quad * 32 + r;
+          if (mr < M) *reinterpret_cast<uint4*>(Y + static_cast<uint64_t>(mr) * N + n0 + col0 + p * 64 + c * 8) = v;
+        }
+        __syncwarp();
       }
     }
   }
@@ -662,30 +711,30 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(ab * C::kBN + col0);
       __nv_bfloat16* yrow = Y + static_cast<uint64_t>(m) * N + n0 + col0;
+      // the whole 128-column slice into registers first, so the accumulator
+      // is handed back to the MMA before the (slower) global stores
+      uint32_t p[128];
 #pragma unroll
-      for (int h = 0; h < 128 / 32; ++h) {
-        uint32_t p[32];
-        tmem_ld_32x32b_x32(taddr + h * 32, p);
-        tmem_wait_ld();
-        if (m < M) {
-#pragma unroll
-          for (int j = 0; j < 32; j += 8) {
-            uint4 v;
-            __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(p[j + 0]), __uint_as_float(p[j + 1]));
-            __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(p[j + 2]), __uint_as_float(p[j + 3]));
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(p[j + 4]), __uint_as_float(p[j + 5]));
-            __nv_bfloat162 h3 = __floats2bfloat162_rn(__uint_as_float(p[j + 6]), __uint_as_float(p[j + 7]));
-            v.x = *reinterpret_cast<uint32_t*>(&h0);
-            v.y = *reinterpret_cast<uint32_t*>(&h1);
-            v.z = *reinterpret_cast<uint32_t*>(&h2);
-            v.w = *reinterpret_cast<uint32_t*>(&h3);
-            *reinterpret_cast<uint4*>(yrow + h * 32 + j) = v;
-          }
-        }
-      }
+      for (int h = 0; h < 128 / 32; ++h) tmem_ld_32x32b_x32(taddr + h * 32, *reinterpret_cast<uint32_t(*)[32]>(&p[h * 32]));
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[tb]);
+      if (m < M) {
+#pragma unroll
+        for (int j = 0; j < 128; j += 8) {
+          uint4 v;
+          __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(p[j + 0]), __uint_as_float(p[j + 1]));
+          __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(p[j + 2]), __uint_as_float(p[j + 3]));
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(p[j + 4]), __uint_as_float(p[j + 5]));
+          __nv_bfloat162 h3 = __floats2bfloat162_rn(__uint_as_float(p[j + 6]), __uint_as_float(p[j + 7]));
+          v.x = *reinterpret_cast<uint32_t*>(&h0);
+          v.y = *reinterpret_cast<uint32_t*>(&h1);
+          v.z = *reinterpret_cast<uint32_t*>(&h2);
+          v.w = *reinterpret_cast<uint32_t*>(&h3);
+          *reinterpret_cast<uint4*>(yrow + j) = v;
+        }
+      }
       ++tile_no;
     }
   }
