@@ -34,6 +34,8 @@ SIGNATURES = {
     "fgfp8_quant_act": (_INT, [_P, _I64, _I64, _I64, _P, _P, _I64, _INT, _P]),
     "fgfp8_gemm": (_INT, [_P, _P, _I64, _P, _P, _P, _I64, _I64, _I64, _INT, _P]),
     "fgfp8_grouped_gemm": (_INT, [_P, _P, _I64, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _INT, _P]),
+    "fgfp8_linear": (_INT, [_P, _I64, _P, _P, _I64, _P, _P, _P, _I64, _I64, _I64, _INT, _P]),
+    "fgfp8_grouped_linear": (_INT, [_P, _I64, _P, _P, _I64, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _INT, _P]),
     "fgfp8_check_device_status": (_INT, [_P]),
 }
 
@@ -90,6 +92,8 @@ fgfp8_quant_weight = _raw("fgfp8_quant_weight")
 fgfp8_quant_act = _raw("fgfp8_quant_act")
 fgfp8_gemm = _raw("fgfp8_gemm")
 fgfp8_grouped_gemm = _raw("fgfp8_grouped_gemm")
+fgfp8_linear = _raw("fgfp8_linear")
+fgfp8_grouped_linear = _raw("fgfp8_grouped_linear")
 fgfp8_check_device_status = _raw("fgfp8_check_device_status")
 
 
@@ -167,6 +171,48 @@ def grouped_gemm(Xq, Xs, Wq, Ws, group_offs, fmt: int, Y=None, stream=None):
     _check(fgfp8_grouped_gemm(Xq.data_ptr(), Xs.data_ptr(), Xs.shape[1], Wq.data_ptr(), Ws.data_ptr(),
                               Y.data_ptr(), group_offs.data_ptr(), E, M_total, N, K, fmt, _stream(stream)),
            "fgfp8_grouped_gemm")
+    return Y
+
+
+def _act_buffers(X, fmt, Xq, Xs, ld_s):
+    import torch
+    M, K = X.shape
+    ld_s = scale_rows(M, fmt) if ld_s is None else ld_s
+    if Xq is None:
+        Xq = torch.empty((M, K), dtype=torch.uint8, device=X.device)
+    if Xs is None:
+        Xs = torch.empty((K // 128, ld_s), dtype=_scale_dtype(fmt), device=X.device)
+    return Xq, Xs, ld_s
+
+
+def linear(X, Wq, Ws, fmt: int, Y=None, Xq=None, Xs=None, ld_s: int | None = None, stream=None):
+    """The W8A8 linear layer Y = X W^T (bf16 [M, N]) from bf16 X [M, K] and the
+    pre-quantized weight: one call that quantizes X into Xq / Xs (allocated
+    here when not given) and runs the GEMM.  Returns Y."""
+    import torch
+    M, K = X.shape
+    N = Wq.shape[0]
+    Xq, Xs, ld_s = _act_buffers(X, fmt, Xq, Xs, ld_s)
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _check(fgfp8_linear(X.data_ptr(), X.stride(0), Xq.data_ptr(), Xs.data_ptr(), ld_s, Wq.data_ptr(), Ws.data_ptr(),
+                        Y.data_ptr(), M, N, K, fmt, _stream(stream)), "fgfp8_linear")
+    return Y
+
+
+def grouped_linear(X, Wq, Ws, group_offs, fmt: int, Y=None, Xq=None, Xs=None, ld_s: int | None = None,
+                   stream=None):
+    """The M-grouped expert layer from bf16 rows X [M_total, K] grouped per
+    expert: quantization and grouped GEMM in one call.  Returns Y."""
+    import torch
+    M_total, K = X.shape
+    E, N, _ = Wq.shape
+    Xq, Xs, ld_s = _act_buffers(X, fmt, Xq, Xs, ld_s)
+    if Y is None:
+        Y = torch.empty((M_total, N), dtype=torch.bfloat16, device=X.device)
+    _check(fgfp8_grouped_linear(X.data_ptr(), X.stride(0), Xq.data_ptr(), Xs.data_ptr(), ld_s, Wq.data_ptr(),
+                                Ws.data_ptr(), Y.data_ptr(), group_offs.data_ptr(), E, M_total, N, K, fmt,
+                                _stream(stream)), "fgfp8_grouped_linear")
     return Y
 
 

@@ -108,6 +108,27 @@ fgfp8_status set_smem(const void* kernel, size_t bytes, int dev) {
   return FGFP8_OK;
 }
 
+// Launch with programmatic stream serialization: the grid may be scheduled
+// while the preceding kernel in the stream is finishing; the kernels wait
+// (griddepcontrol.wait) before touching memory that kernel may write.
+template <typename... KArgs, typename... Args>
+fgfp8_status launch_dependent(void (*kernel)(KArgs...), unsigned grid, unsigned threads, size_t smem,
+                              cudaStream_t stream, const char* what, Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return ok();
+}
+
 fgfp8_status check_launch(const char* what) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, what);
@@ -136,7 +157,7 @@ fgfp8_status check_act_scales(const void* Xs, int64_t ld_s, int64_t M, int fmt) 
 template <int BN, int CW, int FMT, bool kGrouped>
 fgfp8_status launch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
                          void* Y, int64_t M, int64_t N, int64_t K, const int32_t* offs, int E, int64_t b_rows,
-                         cudaStream_t stream, int dev, int sm_count) {
+                         cudaStream_t stream, int dev, int sm_count, int early) {
   using C = fgfp8::GemmCfg<BN, CW>;
   CUtensorMap mA, mB;
   fgfp8_status st = make_map_u8_sw128(&mA, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
@@ -163,17 +184,17 @@ fgfp8_status launch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const 
   const int64_t tiles = ((M + C::kBM - 1) / C::kBM) * (N / BN);
   if (tiles == 0) return ok();
   const int64_t grid = tiles < sm_count ? tiles : sm_count;
-  kernel<<<static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, stream>>>(
-      mA, mB, Xs, static_cast<uint32_t>(ld_s), Ws, reinterpret_cast<__nv_bfloat16*>(Y), static_cast<int>(M),
-      static_cast<int>(N), static_cast<int>(K), offs, E, static_cast<int>(tiles));
-  return check_launch("gemm launch");
+  return launch_dependent(kernel, static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, stream, "gemm launch", mA,
+                          mB, Xs, static_cast<uint32_t>(ld_s), Ws, reinterpret_cast<__nv_bfloat16*>(Y),
+                          static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), offs, E,
+                          static_cast<int>(tiles), early);
 }
 
 // UE8M0 launch with hardware block scaling (persistent, 128 x BN tiles).
 template <int BN, bool kGrouped>
 fgfp8_status launch_gemm_mx(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
                             void* Y, int64_t M, int64_t N, int64_t K, const int32_t* offs, int E, int64_t b_rows,
-                            cudaStream_t stream, int dev, int sm_count) {
+                            cudaStream_t stream, int dev, int sm_count, int early) {
   using C = fgfp8::MxCfg<BN>;
   CUtensorMap mA, mB;
   fgfp8_status st = make_map_u8_sw128(&mA, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
@@ -188,17 +209,17 @@ fgfp8_status launch_gemm_mx(const uint8_t* Xq, const void* Xs, int64_t ld_s, con
   const int64_t tiles = ((M + C::kBM - 1) / C::kBM) * (N / C::kBN);
   if (tiles == 0) return ok();
   const int64_t grid = tiles < sm_count ? tiles : sm_count;
-  kernel<<<static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, stream>>>(
-      mA, mB, reinterpret_cast<const uint8_t*>(Xs), static_cast<uint32_t>(ld_s), reinterpret_cast<const uint8_t*>(Ws),
-      reinterpret_cast<__nv_bfloat16*>(Y), static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), offs, E,
-      static_cast<int>(tiles));
-  return check_launch("block-scaled gemm launch");
+  return launch_dependent(kernel, static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, stream,
+                          "block-scaled gemm launch", mA, mB, reinterpret_cast<const uint8_t*>(Xs),
+                          static_cast<uint32_t>(ld_s), reinterpret_cast<const uint8_t*>(Ws),
+                          reinterpret_cast<__nv_bfloat16*>(Y), static_cast<int>(M), static_cast<int>(N),
+                          static_cast<int>(K), offs, E, static_cast<int>(tiles), early);
 }
 
 template <bool kGrouped>
 fgfp8_status dispatch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws, void* Y,
                            int64_t M, int64_t N, int64_t K, int fmt, const int32_t* offs, int E, int64_t b_rows,
-                           cudaStream_t s, int dev, int sms) {
+                           cudaStream_t s, int dev, int sms, int early) {
   // 128x256 tiles: measured faster per FLOP than 128x128 on B200 even where
   // 128x128 tiles would fill the last wave better (4096^3: 95 us vs 119 us);
   // 128x128 only when N is not a multiple of 256.
@@ -209,16 +230,18 @@ fgfp8_status dispatch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, cons
   constexpr int kWideCW = 128;
   // UE8M0 scales: the tensor core applies them (block-scaled MMA), no promotion.
   if (fmt == FGFP8_SCALE_UE8M0)
-    return wide ? launch_gemm_mx<256, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms)
-                : launch_gemm_mx<128, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms);
-  return wide ? launch_gemm<256, kWideCW, 0, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms)
-              : launch_gemm<128, 64, 0, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms);
+    return wide ? launch_gemm_mx<256, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms, early)
+                : launch_gemm_mx<128, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms, early);
+  return wide ? launch_gemm<256, kWideCW, 0, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms,
+                                                       early)
+              : launch_gemm<128, 64, 0, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms,
+                                                  early);
 }
 
 // Few-token (M <= 64) launch: one CTA per 128 output columns, operands swapped.
 template <int BNT, int FMT>
 fgfp8_status launch_decode(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
-                           void* Y, int64_t M, int64_t N, int64_t K, cudaStream_t stream, int dev) {
+                           void* Y, int64_t M, int64_t N, int64_t K, cudaStream_t stream, int dev, int early) {
   using C = fgfp8::DecodeCfg<BNT>;
   CUtensorMap mX, mW;
   fgfp8_status st = make_map_u8_sw128(&mX, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
@@ -229,18 +252,18 @@ fgfp8_status launch_decode(const uint8_t* Xq, const void* Xs, int64_t ld_s, cons
   auto kernel = fgfp8::gemm_decode_kernel<BNT, FMT>;
   st = set_smem(reinterpret_cast<const void*>(kernel), C::kSmemBytes, dev);
   if (st != FGFP8_OK) return st;
-  kernel<<<static_cast<unsigned>(N / 128), C::kThreads, C::kSmemBytes, stream>>>(
-      mX, mW, Xs, static_cast<uint32_t>(ld_s), Ws, reinterpret_cast<__nv_bfloat16*>(Y), static_cast<int>(M),
-      static_cast<int>(N), static_cast<int>(K));
-  return check_launch("decode gemm launch");
+  return launch_dependent(kernel, static_cast<unsigned>(N / 128), C::kThreads, C::kSmemBytes, stream,
+                          "decode gemm launch", mX, mW, Xs, static_cast<uint32_t>(ld_s), Ws,
+                          reinterpret_cast<__nv_bfloat16*>(Y), static_cast<int>(M), static_cast<int>(N),
+                          static_cast<int>(K), early);
 }
 
 template <int FMT>
 fgfp8_status dispatch_decode(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
-                             void* Y, int64_t M, int64_t N, int64_t K, cudaStream_t s, int dev) {
-  if (M <= 16) return launch_decode<16, FMT>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev);
-  if (M <= 32) return launch_decode<32, FMT>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev);
-  return launch_decode<64, FMT>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev);
+                             void* Y, int64_t M, int64_t N, int64_t K, cudaStream_t s, int dev, int early) {
+  if (M <= 16) return launch_decode<16, FMT>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev, early);
+  if (M <= 32) return launch_decode<32, FMT>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev, early);
+  return launch_decode<64, FMT>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev, early);
 }
 
 fgfp8_status check_gemm_common(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
@@ -263,14 +286,11 @@ fgfp8_status check_gemm_common(const uint8_t* Xq, const void* Xs, int64_t ld_s, 
 
 }  // namespace
 
-extern "C" {
+namespace {
 
-int fgfp8_version(void) { return FGFP8_VERSION; }
-
-const char* fgfp8_last_error_string(void) { return t_last_error.c_str(); }
-
-fgfp8_status fgfp8_quant_act(const void* X, int64_t M, int64_t K, int64_t ldx, uint8_t* Xq, void* Xs, int64_t ld_s,
-                             int fmt, void* stream) {
+// Dynamic 1x128 activation quantization; with dry set, only validates.
+fgfp8_status quant_act_impl(const void* X, int64_t M, int64_t K, int64_t ldx, uint8_t* Xq, void* Xs, int64_t ld_s,
+                            int fmt, void* stream, bool dry) {
   fgfp8_status st = check_fmt(fmt);
   if (st != FGFP8_OK) return st;
   if (M < 0 || K < 0 || ldx < 0) return fail(FGFP8_ERR_INVALID_ARG, "negative size");
@@ -284,6 +304,7 @@ fgfp8_status fgfp8_quant_act(const void* X, int64_t M, int64_t K, int64_t ldx, u
   if (st != FGFP8_OK) return st;
   if (!aligned(X, 16) || ldx % 8 != 0) return fail(FGFP8_ERR_ALIGN, "X must be 16-byte aligned with ldx % 8 == 0");
   if (!aligned(Xq, 16)) return fail(FGFP8_ERR_ALIGN, "Xq must be 16-byte aligned");
+  if (dry) return FGFP8_OK;
   int dev;
   DeviceInfo info;
   st = current_device(&dev, &info);
@@ -308,6 +329,57 @@ fgfp8_status fgfp8_quant_act(const void* X, int64_t M, int64_t K, int64_t ldx, u
                                                                static_cast<uint64_t>(ld_s), kbd);
   return check_launch("quant_act launch");
 }
+
+// Dense block-scaled GEMM; early lets the weight loads start before the wait
+// for the preceding grid; with dry set, only validates.
+fgfp8_status gemm_impl(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws, void* Y,
+                       int64_t M, int64_t N, int64_t K, int fmt, void* stream, int early, bool dry) {
+  if (M == 0 && fmt >= 0 && fmt <= 1 && N >= 0 && K >= 0) return ok();
+  fgfp8_status st = check_gemm_common(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, fmt);
+  if (st != FGFP8_OK) return st;
+  if (dry) return FGFP8_OK;
+  int dev;
+  DeviceInfo info;
+  st = current_device(&dev, &info);
+  if (st != FGFP8_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (M <= 64) {
+    return fmt == FGFP8_SCALE_F32 ? dispatch_decode<0>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev, early)
+                                  : dispatch_decode<1>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev, early);
+  }
+  return dispatch_gemm<false>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, fmt, nullptr, 1, N, s, dev, info.sm_count, early);
+}
+
+// M-grouped expert GEMM; with dry set, only validates.
+fgfp8_status grouped_impl(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws, void* Y,
+                          const int32_t* group_offs, int32_t E, int64_t M_total, int64_t N, int64_t K, int fmt,
+                          void* stream, bool dry) {
+  if (E <= 0) return fail(FGFP8_ERR_INVALID_ARG, "E must be >= 1");
+  if (M_total % 128 != 0) return fail(FGFP8_ERR_SHAPE, "M_total must be a multiple of 128");
+  if (M_total == 0 && fmt >= 0 && fmt <= 1 && N >= 0 && K >= 0) return ok();
+  fgfp8_status st = check_gemm_common(Xq, Xs, ld_s, Wq, Ws, Y, M_total, N, K, fmt);
+  if (st != FGFP8_OK) return st;
+  if (!group_offs) return fail(FGFP8_ERR_INVALID_ARG, "group_offs is NULL");
+  if (!aligned(group_offs, 4)) return fail(FGFP8_ERR_ALIGN, "group_offs must be 4-byte aligned");
+  if (static_cast<int64_t>(E) * N >= (int64_t(1) << 31))
+    return fail(FGFP8_ERR_SHAPE, "E*N must be < 2^31");
+  if (dry) return FGFP8_OK;
+  int dev;
+  DeviceInfo info;
+  st = current_device(&dev, &info);
+  if (st != FGFP8_OK) return st;
+  return dispatch_gemm<true>(Xq, Xs, ld_s, Wq, Ws, Y, M_total, N, K, fmt, group_offs, E,
+                             static_cast<int64_t>(E) * N, reinterpret_cast<cudaStream_t>(stream), dev, info.sm_count, 0);
+}
+
+}  // namespace
+
+extern "C" {
+
+int fgfp8_version(void) { return FGFP8_VERSION; }
+
+const char* fgfp8_last_error_string(void) { return t_last_error.c_str(); }
+
 
 fgfp8_status fgfp8_quant_weight(const void* W, int64_t N, int64_t K, int64_t ldw, uint8_t* Wq, void* Ws, int fmt,
                                 void* stream) {
@@ -342,41 +414,46 @@ fgfp8_status fgfp8_quant_weight(const void* W, int64_t N, int64_t K, int64_t ldw
   return check_launch("quant_weight launch");
 }
 
+
+
+fgfp8_status fgfp8_quant_act(const void* X, int64_t M, int64_t K, int64_t ldx, uint8_t* Xq, void* Xs, int64_t ld_s,
+                             int fmt, void* stream) {
+  return quant_act_impl(X, M, K, ldx, Xq, Xs, ld_s, fmt, stream, false);
+}
+
 fgfp8_status fgfp8_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws, void* Y,
                         int64_t M, int64_t N, int64_t K, int fmt, void* stream) {
-  if (M == 0 && fmt >= 0 && fmt <= 1 && N >= 0 && K >= 0) return ok();
-  fgfp8_status st = check_gemm_common(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, fmt);
-  if (st != FGFP8_OK) return st;
-  int dev;
-  DeviceInfo info;
-  st = current_device(&dev, &info);
-  if (st != FGFP8_OK) return st;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (M <= 64) {
-    return fmt == FGFP8_SCALE_F32 ? dispatch_decode<0>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev)
-                                  : dispatch_decode<1>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev);
-  }
-  return dispatch_gemm<false>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, fmt, nullptr, 1, N, s, dev, info.sm_count);
+  return gemm_impl(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, fmt, stream, 0, false);
 }
 
 fgfp8_status fgfp8_grouped_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
                                 void* Y, const int32_t* group_offs, int32_t E, int64_t M_total, int64_t N, int64_t K,
                                 int fmt, void* stream) {
-  if (E <= 0) return fail(FGFP8_ERR_INVALID_ARG, "E must be >= 1");
-  if (M_total % 128 != 0) return fail(FGFP8_ERR_SHAPE, "M_total must be a multiple of 128");
-  if (M_total == 0 && fmt >= 0 && fmt <= 1 && N >= 0 && K >= 0) return ok();
-  fgfp8_status st = check_gemm_common(Xq, Xs, ld_s, Wq, Ws, Y, M_total, N, K, fmt);
+  return grouped_impl(Xq, Xs, ld_s, Wq, Ws, Y, group_offs, E, M_total, N, K, fmt, stream, false);
+}
+
+fgfp8_status fgfp8_linear(const void* X, int64_t ldx, uint8_t* Xq, void* Xs, int64_t ld_s, const uint8_t* Wq,
+                          const void* Ws, void* Y, int64_t M, int64_t N, int64_t K, int fmt, void* stream) {
+  fgfp8_status st = quant_act_impl(X, M, K, ldx, Xq, Xs, ld_s, fmt, stream, true);
   if (st != FGFP8_OK) return st;
-  if (!group_offs) return fail(FGFP8_ERR_INVALID_ARG, "group_offs is NULL");
-  if (!aligned(group_offs, 4)) return fail(FGFP8_ERR_ALIGN, "group_offs must be 4-byte aligned");
-  if (static_cast<int64_t>(E) * N >= (int64_t(1) << 31))
-    return fail(FGFP8_ERR_SHAPE, "E*N must be < 2^31");
-  int dev;
-  DeviceInfo info;
-  st = current_device(&dev, &info);
+  st = gemm_impl(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, fmt, stream, 1, true);
   if (st != FGFP8_OK) return st;
-  return dispatch_gemm<true>(Xq, Xs, ld_s, Wq, Ws, Y, M_total, N, K, fmt, group_offs, E,
-                             static_cast<int64_t>(E) * N, reinterpret_cast<cudaStream_t>(stream), dev, info.sm_count);
+  st = quant_act_impl(X, M, K, ldx, Xq, Xs, ld_s, fmt, stream, false);
+  if (st != FGFP8_OK) return st;
+  // the quantizer writes only Xq and Xs: the GEMM may request weight tiles early
+  return gemm_impl(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, fmt, stream, 1, false);
+}
+
+fgfp8_status fgfp8_grouped_linear(const void* X, int64_t ldx, uint8_t* Xq, void* Xs, int64_t ld_s, const uint8_t* Wq,
+                                  const void* Ws, void* Y, const int32_t* group_offs, int32_t E, int64_t M_total,
+                                  int64_t N, int64_t K, int fmt, void* stream) {
+  fgfp8_status st = quant_act_impl(X, M_total, K, ldx, Xq, Xs, ld_s, fmt, stream, true);
+  if (st != FGFP8_OK) return st;
+  st = grouped_impl(Xq, Xs, ld_s, Wq, Ws, Y, group_offs, E, M_total, N, K, fmt, stream, true);
+  if (st != FGFP8_OK) return st;
+  st = quant_act_impl(X, M_total, K, ldx, Xq, Xs, ld_s, fmt, stream, false);
+  if (st != FGFP8_OK) return st;
+  return grouped_impl(Xq, Xs, ld_s, Wq, Ws, Y, group_offs, E, M_total, N, K, fmt, stream, false);
 }
 
 fgfp8_status fgfp8_check_device_status(void* stream) {

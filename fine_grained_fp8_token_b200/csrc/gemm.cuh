@@ -127,11 +127,21 @@ __device__ __forceinline__ int find_expert(const int32_t* __restrict__ offs, int
 
 // TMA producer (one thread): per K block, a kABytes tile of operand A (rows
 // a_row.., box from tmA) and a kBBytes tile of operand B into ring slot
-// kb % kStages; waits for the slot to be released by the MMA first.  Before
-// returning it waits for every copy it issued to land.
+// kb % kStages; waits for the slot to be released by the MMA first.  With
+// early_a, the A tiles of the first kStages K blocks are requested before the
+// wait for the preceding grid (A must not be written by it); every other
+// load follows that wait.  Before returning it waits for every copy it
+// issued to land.
 template <int kStages, uint32_t kABytes, uint32_t kBBytes>
 __device__ __forceinline__ void produce_tiles(const CUtensorMap* tmA, int a_row, const CUtensorMap* tmB, int b_row,
-                                              int KB, uint8_t* sA, uint8_t* sB, uint64_t* full, uint64_t* empty) {
+                                              int KB, uint8_t* sA, uint8_t* sB, uint64_t* full, uint64_t* empty,
+                                              bool early_a) {
+  const int pre = early_a ? (KB < kStages ? KB : kStages) : 0;
+  for (int kb = 0; kb < pre; ++kb) {
+    mbar_arrive_expect_tx(&full[kb], kABytes + kBBytes);
+    tma_load_2d(sA + kb * kABytes, tmA, &full[kb], kb * 128, a_row);
+  }
+  griddep_wait();
   int issued = 0;
   for (int kb = 0; kb < KB; ++kb) {
     const int s = kb % kStages;
@@ -140,8 +150,10 @@ __device__ __forceinline__ void produce_tiles(const CUtensorMap* tmA, int a_row,
       record_status(kDevTimeoutProducer);
       break;
     }
-    mbar_arrive_expect_tx(&full[s], kABytes + kBBytes);
-    tma_load_2d(sA + s * kABytes, tmA, &full[s], kb * 128, a_row);
+    if (kb >= pre) {
+      mbar_arrive_expect_tx(&full[s], kABytes + kBBytes);
+      tma_load_2d(sA + s * kABytes, tmA, &full[s], kb * 128, a_row);
+    }
     tma_load_2d(sB + s * kBBytes, tmB, &full[s], kb * 128, b_row);
     issued = kb + 1;
   }
@@ -192,7 +204,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
     gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const void* __restrict__ Xs, uint32_t ld_s, const void* __restrict__ Ws,
                             __nv_bfloat16* __restrict__ Y, int M, int N, int K,
-                            const int32_t* __restrict__ group_offs, int E, int num_tiles) {
+                            const int32_t* __restrict__ group_offs, int E, int num_tiles, int early_b) {
   using C = GemmCfg<BN, CW>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -254,11 +266,28 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Dependency on the preceding grid (programmatic launch): the producer may
+  // request the first weight tiles before it; every other access follows it.
+  if (threadIdx.x != 0) griddep_wait();
 
   if (warp < 4) {
     if (C::kRegSplit) setmaxnreg_dec<C::kRegsLow>();
     if (warp == 0 && lane == 0) {
       // ================= TMA producer
+      // early_b (dense): the weight tiles of the first tile's first kStages K
+      // blocks are requested before the wait (the weights must not be
+      // written by the preceding grid).
+      int pre = 0;
+      if (!kGrouped && early_b && static_cast<int>(blockIdx.x) < num_tiles) {
+        int m0, n0, expert;
+        coords(blockIdx.x, m0, n0, expert);
+        pre = KB < C::kStages ? KB : C::kStages;
+        for (int kb = 0; kb < pre; ++kb) {
+          mbar_arrive_expect_tx(&full[kb], C::kStageBytes);
+          tma_load_2d(sB + kb * C::kBBytes, &tmB, &full[kb], kb * C::kBK, n0);
+        }
+      }
+      griddep_wait();
       uint32_t it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
@@ -276,9 +305,11 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+          if (it >= static_cast<uint32_t>(pre)) {
+            mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+            tma_load_2d(sB + s * C::kBBytes, &tmB, &full[s], kb * C::kBK, b_row);
+          }
           tma_load_2d(sA + s * C::kABytes, &tmA, &full[s], kb * C::kBK, m0);
-          tma_load_2d(sB + s * C::kBBytes, &tmB, &full[s], kb * C::kBK, b_row);
         }
       }
       // every copy issued must land before the CTA may exit
@@ -510,7 +541,7 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
     gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const uint8_t* __restrict__ Xs, uint32_t ld_s, const uint8_t* __restrict__ Ws,
                    __nv_bfloat16* __restrict__ Y, int M, int N, int K, const int32_t* __restrict__ group_offs,
-                   int E, int num_tiles) {
+                   int E, int num_tiles, int early_b) {
   using C = MxCfg<BN>;
   static_assert(C::kSfCol + 2 * C::kSfColsPerKb <= C::kTmemCols, "TMEM columns");
   extern __shared__ uint8_t smem_raw[];
@@ -570,8 +601,28 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  // Dependency on the preceding grid (programmatic launch): the producer may
+  // request the first weight tiles before it; every other access follows it.
+  if (warp != 0) griddep_wait();
+
   if (warp == 0) {
     // ================= producer: TMA (lane 0) + scale rows (all lanes)
+    // early_b (dense): the weight tiles of the first tile's first kStages K
+    // blocks are requested before the wait (the weights must not be written
+    // by the preceding grid).
+    int pre = 0;
+    if (!kGrouped && early_b && static_cast<int>(blockIdx.x) < num_tiles) {
+      int m0, n0, expert;
+      coords(blockIdx.x, m0, n0, expert);
+      pre = KB < C::kStages ? KB : C::kStages;
+      if (lane == 0) {
+        for (int kb = 0; kb < pre; ++kb) {
+          mbar_arrive_expect_tx(&full[kb], C::kStageBytes);
+          tma_load_2d(sB + kb * C::kBBytes, &tmB, &full[kb], kb * C::kBK, n0);
+        }
+      }
+    }
+    griddep_wait();
     uint32_t it = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
@@ -609,9 +660,11 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
             break;
           }
           if (lane == 0) {
-            mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+            if (it >= static_cast<uint32_t>(pre)) {
+              mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+              tma_load_2d(sB + s * C::kBBytes, &tmB, &full[s], kb * C::kBK, expert * N + n0);
+            }
             tma_load_2d(sA + s * C::kABytes, &tmA, &full[s], kb * C::kBK, m0);
-            tma_load_2d(sB + s * C::kBBytes, &tmB, &full[s], kb * C::kBK, expert * N + n0);
           }
           // scale rows in the TMEM scale layout: lane l holds rows l + 32 j,
           // each byte repeated for the four 32-element K slices
@@ -770,7 +823,7 @@ template <int BNT, int FMT>
 __global__ void __launch_bounds__(DecodeCfg<BNT>::kThreads, 1)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                        const void* __restrict__ Xs, uint32_t ld_s, const void* __restrict__ Ws,
-                       __nv_bfloat16* __restrict__ Y, int M, int N, int K) {
+                       __nv_bfloat16* __restrict__ Y, int M, int N, int K, int early_w) {
   using C = DecodeCfg<BNT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -813,9 +866,12 @@ __global__ void __launch_bounds__(DecodeCfg<BNT>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  // Dependency on the preceding grid (programmatic launch): the producer may
+  // request the first weight tiles before it; every other access follows it.
+  if (threadIdx.x != 0) griddep_wait();
   if (warp == 0) {
     if (lane == 0)
-      produce_tiles<C::kStages, C::kABytes, C::kBBytes>(&tmW, n0, &tmX, 0, KB, sW, sX, full, empty);
+      produce_tiles<C::kStages, C::kABytes, C::kBBytes>(&tmW, n0, &tmX, 0, KB, sW, sX, full, empty, early_w != 0);
   } else if (warp == 1) {
     if (lane == 0)
       issue_mmas<C::kStages, C::kABytes, C::kBBytes, BNT, C::kNumBuf>(smem_u32(sW), smem_u32(sX), KB, tmem_base,

@@ -22,6 +22,8 @@
 #include <cuda_fp8.h>
 #include <cstdint>
 
+#include "ptx.cuh"
+
 namespace fgfp8 {
 
 constexpr int kGroup = 128;
@@ -138,6 +140,9 @@ template <int FMT, int UNROLL>
 __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restrict__ X, uint32_t M, uint32_t K,
                                                         uint64_t ldx, uint8_t* __restrict__ Xq,
                                                         void* __restrict__ Xs, uint64_t ld_s, FastDiv kb_div) {
+  // a GEMM launched after this kernel with programmatic serialization may be
+  // scheduled now; it waits for this grid's completion before reading Xq / Xs
+  griddep_launch_dependents();
   const uint32_t total = M * kb_div.d;
   const uint32_t lane = threadIdx.x & 31u;
   const uint32_t sub = lane & 7u;

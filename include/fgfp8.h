@@ -111,6 +111,9 @@ fgfp8_status fgfp8_quant_act(const void* X, int64_t M, int64_t K, int64_t ldx, u
  *   Y             bf16 [M, N] row-major (row stride N), 16-byte aligned.
  * K % 128 == 0, N % 128 == 0, M >= 0 arbitrary (M == 0 is a no-op).
  * M, N, K < 2^31.
+ * The GEMM kernels are launched with programmatic stream serialization: they
+ * may be scheduled while the preceding kernel in `stream` finishes, and wait
+ * for its completion before their first access to global memory.
  */
 fgfp8_status fgfp8_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
                         void* Y, int64_t M, int64_t N, int64_t K, int fmt, void* stream);
@@ -135,6 +138,29 @@ fgfp8_status fgfp8_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const u
 fgfp8_status fgfp8_grouped_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq,
                                 const void* Ws, void* Y, const int32_t* group_offs, int32_t E,
                                 int64_t M_total, int64_t N, int64_t K, int fmt, void* stream);
+
+/*
+ * The whole W8A8 linear layer: fgfp8_quant_act of X into the caller's Xq /
+ * Xs buffers followed by fgfp8_gemm ("Fine-grained FP8", introduction and
+ * "DeepGEMM fast path": activations are quantized on the fly, weights are
+ * pre-quantized).  Arguments mean what they mean for those two calls; every
+ * argument of both is validated before anything is launched, so on an error
+ * nothing has been written.  The GEMM is launched as a programmatic
+ * dependent of the quantizer and may start streaming Wq while the quantizer
+ * runs: the quantizer writes only Xq and Xs, and it starts only after all
+ * earlier work on `stream` has completed.  Y equals fgfp8_gemm's.
+ */
+fgfp8_status fgfp8_linear(const void* X, int64_t ldx, uint8_t* Xq, void* Xs, int64_t ld_s, const uint8_t* Wq,
+                          const void* Ws, void* Y, int64_t M, int64_t N, int64_t K, int fmt, void* stream);
+
+/*
+ * The M-grouped expert layer: fgfp8_quant_act of the expert-grouped rows X
+ * [M_total, K] followed by fgfp8_grouped_gemm, with the same validation-first
+ * behaviour as fgfp8_linear.
+ */
+fgfp8_status fgfp8_grouped_linear(const void* X, int64_t ldx, uint8_t* Xq, void* Xs, int64_t ld_s,
+                                  const uint8_t* Wq, const void* Ws, void* Y, const int32_t* group_offs,
+                                  int32_t E, int64_t M_total, int64_t N, int64_t K, int fmt, void* stream);
 
 /*
  * Synchronizes `stream`, then reads and clears the device status word that

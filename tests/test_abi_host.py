@@ -101,6 +101,27 @@ def test_grouped_gemm_validation():
     assert f(A, A, 256, A, A, A, A, 4, 0, 256, 256, 1, None) == OK            # empty
 
 
+def test_linear_validates_both_halves_first():
+    """fgfp8_linear checks the quantizer's and the GEMM's arguments before it
+    launches anything: a bad GEMM argument is reported even though the
+    quantizer's arguments are valid (so no kernel has written Xq / Xs)."""
+    f = fg.fgfp8_linear
+    # X, ldx, Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, fmt, stream
+    assert f(A, 256, A, A, 4, A, A, A, 4, 256, 100, 0, None) == SHAPE      # K % 128 (both)
+    assert f(A, 128, A, A, 4, A, A, A, 4, 256, 256, 0, None) == SHAPE      # ldx < K (quantizer)
+    assert f(A, 256, A, A, 4, A, A, A, 4, 200, 256, 0, None) == SHAPE      # N % 128 (GEMM only)
+    assert f(A, 256, A, A, 4, A, A, A + 8, 4, 256, 256, 0, None) == ALIGN  # Y (GEMM only)
+    assert f(A, 256, A, A, 4, 0, A, A, 4, 256, 256, 0, None) == INVALID    # NULL Wq (GEMM only)
+    assert f(A, 256, A, A, 4, A, A, A, 4, 256, 256, 3, None) == INVALID    # fmt
+    assert f(A, 256, A, A, 4, A, A, A, 0, 256, 256, 0, None) == OK         # empty
+    g = fg.fgfp8_grouped_linear
+    # X, ldx, Xq, Xs, ld_s, Wq, Ws, Y, offs, E, M_total, N, K, fmt, stream
+    assert g(A, 256, A, A, 256, A, A, A, A, 0, 256, 256, 256, 1, None) == INVALID   # E
+    assert g(A, 256, A, A, 256, A, A, A, A, 4, 200, 256, 256, 1, None) == SHAPE     # M_total % 128
+    assert g(A, 256, A, A, 256, A, A, A, 0, 4, 256, 256, 256, 1, None) == INVALID   # NULL offsets
+    assert g(A, 256, A, A, 256, A, A, A, A, 4, 0, 256, 256, 1, None) == OK          # empty
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the behaviour without a GPU")
 def test_valid_call_without_gpu_fails_loudly():
     """No CPU fallback: a well-formed request on a machine without an
@@ -108,5 +129,6 @@ def test_valid_call_without_gpu_fails_loudly():
     assert fg.fgfp8_quant_act(A, 4, 256, 256, A, A, 4, 0, None) == CUDA
     assert "cuda" in fg.fgfp8_last_error_string().lower()
     assert fg.fgfp8_gemm(A, A, 4, A, A, A, 4, 256, 256, 0, None) == CUDA
+    assert fg.fgfp8_linear(A, 256, A, A, 4, A, A, A, 4, 256, 256, 0, None) == CUDA
     with pytest.raises(fg.FGFP8Error):
         fg._check(fg.fgfp8_quant_weight(A, 128, 256, 256, A, A, 0, None), "quant_weight")

@@ -195,3 +195,75 @@ def test_grouped_gemm_bad_offsets_reported(dev):
     assert ei.value.status == 7
     assert (Y[:128].float() == 0).all() and (Y[128:].float() == 7).all()
     fg.check_device_status()       # the status word was cleared
+
+
+# ---------------------------------------------------------------- one-call linear layer
+LINEAR_CASES = [(300, 640, 2048, F32), (513, 512, 4096, UE8M0), (1, 1280, 7168, UE8M0), (64, 256, 1024, F32),
+                (33, 384, 512, F32), (4096, 4096, 4096, F32)]
+
+
+@pytest.mark.parametrize("M,N,K,fmt", LINEAR_CASES)
+def test_linear_equals_quant_then_gemm(dev, M, N, K, fmt):
+    """fgfp8_linear (quantizer + GEMM launched as its programmatic dependent,
+    weight tiles requested early) gives bit-for-bit the codes, scales and
+    output of the two separate calls."""
+    cfg = workloads.scaled_linear(workloads.TINY, M=M, N=N, K=K, seed=11 * M + N)
+    X, W = workloads.linear_inputs(cfg, device=dev)
+    Wq, Ws = fg.quant_weight(W, fmt)
+    Xq1, Xs1 = fg.quant_act(X, fmt)
+    Y1 = fg.gemm(Xq1, Xs1, Wq, Ws, fmt)
+    Xq2 = torch.empty_like(Xq1)
+    Xs2 = torch.empty_like(Xs1)
+    Y2 = fg.linear(X, Wq, Ws, fmt, Xq=Xq2, Xs=Xs2)
+    fg.check_device_status()
+    assert torch.equal(Xq1, Xq2)
+    assert torch.equal(Xs1[:, :M].contiguous().view(torch.uint8), Xs2[:, :M].contiguous().view(torch.uint8))
+    assert torch.equal(Y1, Y2)
+
+
+@pytest.mark.parametrize("M,N,K,fmt", [(129, 384, 1024, F32), (7, 256, 384, UE8M0)])
+def test_linear_oracle_parity(dev, M, N, K, fmt):
+    cfg = workloads.scaled_linear(workloads.TINY, M=M, N=N, K=K, seed=5 * M + K)
+    X, W = workloads.linear_inputs(cfg)
+    Wq, Ws = fg.quant_weight(W.to(dev), fmt)
+    Y = fg.linear(X.to(dev), Wq, Ws, fmt)
+    fg.check_device_status()
+    Y_ref, S = oracle_linear(bits16(X), bits16(W), fmt)
+    assert_gemm_close(y_to_f64(Y), Y_ref, S, f"linear {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("M", [2, 300])
+def test_linear_back_to_back_weight_updates(dev, M):
+    """Weights re-quantized between layer calls on the same stream, with no
+    host synchronisation: every call sees the weights written just before it
+    (the early weight loads never overtake the preceding fgfp8_quant_weight)."""
+    N, K = 512, 1024
+    g = torch.Generator(device=dev).manual_seed(3)
+    X = (torch.randn((M, K), generator=g, device=dev)).to(torch.bfloat16)
+    Ws_list = [(torch.randn((N, K), generator=g, device=dev) * 0.02).to(torch.bfloat16) for _ in range(6)]
+    Wq = torch.empty((N, K), dtype=torch.uint8, device=dev)
+    Wsc = torch.empty((N // 128, K // 128), dtype=torch.float32, device=dev)
+    outs = []
+    for W in Ws_list:
+        fg.quant_weight(W, F32, Wq=Wq, Ws=Wsc)
+        outs.append(fg.linear(X, Wq, Wsc, F32))
+    fg.check_device_status()
+    for W, Y in zip(Ws_list, outs):
+        Wq_i, Ws_i = fg.quant_weight(W, F32)
+        Xq, Xs = fg.quant_act(X, F32)
+        assert torch.equal(Y, fg.gemm(Xq, Xs, Wq_i, Ws_i, F32))
+
+
+@pytest.mark.parametrize("fmt", [UE8M0, F32])
+def test_grouped_linear_equals_two_calls(dev, fmt):
+    cfg = workloads.scaled_moe(workloads.MOE, E=9, N=256, K=512, tokens=300, topk=3, fmt=fmt)
+    r, X, Y1 = build_moe(cfg, dev)
+    Wq = torch.empty((cfg.E, cfg.N, cfg.K), dtype=torch.uint8, device=dev)
+    Ws = torch.empty((cfg.E, cfg.N // 128, cfg.K // 128), dtype=torch.float32 if fmt == F32 else torch.uint8,
+                     device=dev)
+    for e in range(cfg.E):
+        fg.quant_weight(workloads.moe_expert_weight(cfg, e, device=dev), fmt, Wq=Wq[e], Ws=Ws[e])
+    offs = torch.as_tensor(r.group_offs, device=dev)
+    Y2 = fg.grouped_linear(X, Wq, Ws, offs, fmt)
+    fg.check_device_status()
+    assert torch.equal(Y1, Y2)
