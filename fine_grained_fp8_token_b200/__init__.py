@@ -36,6 +36,7 @@ SIGNATURES = {
     "fgfp8_grouped_gemm": (_INT, [_P, _P, _I64, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _INT, _P]),
     "fgfp8_linear": (_INT, [_P, _I64, _P, _P, _I64, _P, _P, _P, _I64, _I64, _I64, _INT, _P]),
     "fgfp8_grouped_linear": (_INT, [_P, _I64, _P, _P, _I64, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _INT, _P]),
+    "fgfp8_linear_noalloc": (_INT, [_P, _I64, _P, _P, _P, _I64, _I64, _I64, _INT, _P]),
     "fgfp8_check_device_status": (_INT, [_P]),
 }
 
@@ -94,6 +95,7 @@ fgfp8_gemm = _raw("fgfp8_gemm")
 fgfp8_grouped_gemm = _raw("fgfp8_grouped_gemm")
 fgfp8_linear = _raw("fgfp8_linear")
 fgfp8_grouped_linear = _raw("fgfp8_grouped_linear")
+fgfp8_linear_noalloc = _raw("fgfp8_linear_noalloc")
 fgfp8_check_device_status = _raw("fgfp8_check_device_status")
 
 

@@ -374,6 +374,38 @@ fgfp8_status grouped_impl(const uint8_t* Xq, const void* Xs, int64_t ld_s, const
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Static scratch of fgfp8_linear_noalloc: the quantized activations (codes,
+// then scales) of one call live here instead of in caller-allocated buffers.
+// Every device that loads this library holds FGFP8_NOALLOC_SCRATCH_BYTES of
+// it until the process exits.  Host code must not pass the symbol itself to
+// a kernel (on the host it names a stand-in object, not device memory): the
+// device address comes from cudaGetSymbolAddress, once per device.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t g_noalloc_scratch[FGFP8_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of g_noalloc_scratch on the current device `dev`, looked up
+// on the first call for that device and cached.  A failed lookup is reported
+// and retried on the next call.
+fgfp8_status noalloc_scratch(int dev, uint8_t** out) {
+  static std::mutex mu;
+  static uint8_t* addr[kMaxDevices] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the static scratch");
+    if (!p || !aligned(p, 256)) return fail(FGFP8_ERR_CUDA, "the static scratch has no 256-byte aligned address");
+    addr[dev] = static_cast<uint8_t*>(p);
+  }
+  *out = addr[dev];
+  return FGFP8_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 int fgfp8_version(void) { return FGFP8_VERSION; }
@@ -454,6 +486,46 @@ fgfp8_status fgfp8_grouped_linear(const void* X, int64_t ldx, uint8_t* Xq, void*
   st = quant_act_impl(X, M_total, K, ldx, Xq, Xs, ld_s, fmt, stream, false);
   if (st != FGFP8_OK) return st;
   return grouped_impl(Xq, Xs, ld_s, Wq, Ws, Y, group_offs, E, M_total, N, K, fmt, stream, false);
+}
+
+fgfp8_status fgfp8_linear_noalloc(const void* X, int64_t ldx, const uint8_t* Wq, const void* Ws, void* Y,
+                                  int64_t M, int64_t N, int64_t K, int fmt, void* stream) {
+  // Everything that can be checked without a device comes first, so an
+  // oversized request is rejected before any CUDA call.
+  fgfp8_status st = check_fmt(fmt);
+  if (st != FGFP8_OK) return st;
+  if (M < 0 || N < 0 || K < 0 || ldx < 0) return fail(FGFP8_ERR_INVALID_ARG, "negative size");
+  if (K == 0 || K % 128 != 0) return fail(FGFP8_ERR_SHAPE, "K must be a positive multiple of 128");
+  if (N == 0 || N % 128 != 0) return fail(FGFP8_ERR_SHAPE, "N must be a positive multiple of 128");
+  if (M == 0) return ok();
+  const int64_t ld_s = (M + 15) / 16 * 16;              // valid for both scale formats
+  const int64_t scale_bytes = (fmt == FGFP8_SCALE_F32) ? 4 : 1;
+  const int64_t limit = static_cast<int64_t>(FGFP8_NOALLOC_SCRATCH_BYTES);
+  if (M > limit || K > limit) return fail(FGFP8_ERR_SHAPE, "M or K exceeds the static scratch");
+  const int64_t codes = (M * K + 255) / 256 * 256;      // Xq, then Xs at a 256-byte boundary
+  const int64_t need = codes + (K / 128) * ld_s * scale_bytes;
+  if (need > limit)
+    return fail(FGFP8_ERR_SHAPE, "M x K too large for the static scratch: the quantized activations need " +
+                                     std::to_string(need) + " bytes, the limit is " + std::to_string(limit) +
+                                     " (FGFP8_NOALLOC_SCRATCH_BYTES); use fgfp8_linear with caller buffers");
+  if (!X || !Wq || !Ws || !Y) return fail(FGFP8_ERR_INVALID_ARG, "X, Wq, Ws or Y is NULL");
+  int dev;
+  DeviceInfo info;
+  st = current_device(&dev, &info);
+  if (st != FGFP8_OK) return st;
+  uint8_t* scratch = nullptr;
+  st = noalloc_scratch(dev, &scratch);
+  if (st != FGFP8_OK) return st;
+  uint8_t* Xq = scratch;
+  void* Xs = scratch + codes;
+  // the same validation-first sequence as fgfp8_linear, on the scratch buffers
+  st = quant_act_impl(X, M, K, ldx, Xq, Xs, ld_s, fmt, stream, true);
+  if (st != FGFP8_OK) return st;
+  st = gemm_impl(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, fmt, stream, 1, true);
+  if (st != FGFP8_OK) return st;
+  st = quant_act_impl(X, M, K, ldx, Xq, Xs, ld_s, fmt, stream, false);
+  if (st != FGFP8_OK) return st;
+  return gemm_impl(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, fmt, stream, 1, false);
 }
 
 fgfp8_status fgfp8_check_device_status(void* stream) {

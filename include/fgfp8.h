@@ -162,6 +162,42 @@ fgfp8_status fgfp8_grouped_linear(const void* X, int64_t ldx, uint8_t* Xq, void*
                                   const uint8_t* Wq, const void* Ws, void* Y, const int32_t* group_offs,
                                   int32_t E, int64_t M_total, int64_t N, int64_t K, int fmt, void* stream);
 
+/* Size of the static scratch of fgfp8_linear_noalloc: 32 MiB per device. */
+#define FGFP8_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * fgfp8_linear without the Xq / Xs buffers, for callers that cannot allocate
+ * device memory.  The source documentation has no counterpart to this call;
+ * it exists for hosts such as a plugin that receives only its input and
+ * output buffers from a framework that owns all device memory, a
+ * latency-critical loop that must not call cudaMalloc (which can synchronize
+ * the device), or a process whose memory pool is sized once at start-up and
+ * refuses further allocations.
+ *
+ * The quantized activations live in one scratch array that the library
+ * reserves statically on every device that loads it (FGFP8_NOALLOC_SCRATCH_BYTES,
+ * held until the process exits).  The codes take M*K bytes rounded up to 256,
+ * followed by the scales: (K/128) * round_up(M, 16) * (4 for F32, 1 for
+ * UE8M0) bytes.  A request whose total exceeds FGFP8_NOALLOC_SCRATCH_BYTES
+ * returns FGFP8_ERR_SHAPE before any CUDA call (for example M = 4096 tokens
+ * fits for K = 4096, M = 8192 does not).
+ *   X, ldx       bf16 [M, K] as for fgfp8_quant_act.
+ *   Wq, Ws, fmt  the pre-quantized weight as for fgfp8_gemm.
+ *   Y            bf16 [M, N], 16-byte aligned.
+ * Y equals fgfp8_linear's for the same arguments.
+ *
+ * This call allocates nothing, through CUDA or any library.  Its first call
+ * on a device looks up the scratch array's device address (with that device
+ * current) and keeps it; make that first call before any stream capture on
+ * the device.  Every call on a device shares the same array and leaves its
+ * contents behind; each call writes every byte it later reads, so nothing
+ * needs clearing between calls.  Calls whose kernels overlap on the GPU
+ * (different streams, or different host threads, without ordering between
+ * them) race on the array and give wrong results: order them on one stream.
+ */
+fgfp8_status fgfp8_linear_noalloc(const void* X, int64_t ldx, const uint8_t* Wq, const void* Ws, void* Y, int64_t M,
+                                  int64_t N, int64_t K, int fmt, void* stream);
+
 /*
  * Synchronizes `stream`, then reads and clears the device status word that
  * the kernels set when they give up.  It returns FGFP8_OK,
