@@ -11,10 +11,11 @@
 //               -> fp32), four K=32 steps per K block, into one of two TMEM
 //               partial buffers (ping-pong), then commits to the slot's
 //               "empty" barrier and the buffer's "full" barrier;
-//   warps 2..   promotion: each thread owns one output row and 128 columns; it
+//   warps 4..   promotion: each thread owns one output row and CW columns; it
 //               loads the block partial from TMEM, multiplies by the product
-//               of the two block scales and accumulates in fp32 registers, so
-//               the MMA of block kb+1 overlaps the promotion of block kb.
+//               of the two block scales and accumulates in fp32 registers
+//               (packed fp32x2 FMAs), so the MMA of block kb+1 overlaps the
+//               promotion of block kb.
 // After the last K block each thread rounds its 128 accumulators to bf16
 // (round-to-nearest-even) and stores them.
 //
@@ -71,8 +72,6 @@ struct GemmCfg {
   static constexpr bool kRegSplit = true;
   static constexpr int kRegsLow = 24;
   static constexpr int kRegsHigh = ((kThreads * kLaunchRegs - 128 * kRegsLow) / (kThreads - 128)) & ~7;
-  // columns loaded per tcgen05.wait::ld in the promotion loop
-  static constexpr int kPerWait = (CW >= 128) ? 64 : 16;
 };
 
 template <int N>
@@ -397,9 +396,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
         for (int d = 0; d < kScaleAhead; ++d) fetch(d, m, live, ws_row, ra[d], rw[d]);
       }
 
-      float acc[CW];
+      // fp32 accumulators as pairs: columns 2j, 2j+1 in acc2[j]
+      float2 acc2[CW / 2];
 #pragma unroll
-      for (int j = 0; j < CW; ++j) acc[j] = 0.0f;
+      for (int j = 0; j < CW / 2; ++j) acc2[j] = make_float2(0.0f, 0.0f);
       for (int kb0 = 0; kb0 < KB && ok; kb0 += kScaleAhead) {
 #pragma unroll
         for (int d = 0; d < kScaleAhead; ++d) {
@@ -416,23 +416,27 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
           }
           tc_fence_after();
           const uint32_t taddr = lane_base + static_cast<uint32_t>(buf * BN);
+          // Two halves of CW/2 columns, each one TMEM load round trip and
+          // packed fp32x2 FMAs (fma.rn per element, as a scalar FMA).  The
+          // buffer is handed back as soon as the second half is in registers;
+          // that half's FMAs run while the next MMA fills the buffer.
+          constexpr int kHalf = CW / 2;
+          const float2 sc2 = make_float2(sc, sc);
+          uint32_t p[kHalf];
+          tmem_ld_cols<kHalf>(taddr, p);
+          tmem_wait_ld();
 #pragma unroll
-          for (int h = 0; h < CW / C::kPerWait; ++h) {
-            uint32_t p[C::kPerWait];
-            if (C::kPerWait == 64) {
-              tmem_ld_32x32b_x32(taddr + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&p[0]));
-              tmem_ld_32x32b_x32(taddr + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&p[C::kPerWait / 2]));
-            } else {
-              tmem_ld_32x32b_x16(taddr + h * 16, *reinterpret_cast<uint32_t(*)[16]>(&p[0]));
-            }
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < C::kPerWait; ++j)
-              acc[h * C::kPerWait + j] = __fmaf_rn(__uint_as_float(p[j]), sc, acc[h * C::kPerWait + j]);
-          }
+          for (int j = 0; j < kHalf / 2; ++j)
+            acc2[j] = __ffma2_rn(make_float2(__uint_as_float(p[2 * j]), __uint_as_float(p[2 * j + 1])), sc2, acc2[j]);
+          tmem_ld_cols<kHalf>(taddr + kHalf, p);
+          tmem_wait_ld();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&tempty[buf]);
+#pragma unroll
+          for (int j = 0; j < kHalf / 2; ++j)
+            acc2[kHalf / 2 + j] =
+                __ffma2_rn(make_float2(__uint_as_float(p[2 * j]), __uint_as_float(p[2 * j + 1])), sc2, acc2[kHalf / 2 + j]);
           ++bt;
         }
       }
@@ -465,10 +469,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
         for (int c = 0; c < 8; ++c) {
           const int j = p * 64 + c * 8;
           uint4 v;
-          __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[j + 0], acc[j + 1]);
-          __nv_bfloat162 h1 = __floats2bfloat162_rn(acc[j + 2], acc[j + 3]);
-          __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[j + 4], acc[j + 5]);
-          __nv_bfloat162 h3 = __floats2bfloat162_rn(acc[j + 6], acc[j + 7]);
+          __nv_bfloat162 h0 = __floats2bfloat162_rn(acc2[j / 2 + 0].x, acc2[j / 2 + 0].y);
+          __nv_bfloat162 h1 = __floats2bfloat162_rn(acc2[j / 2 + 1].x, acc2[j / 2 + 1].y);
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(acc2[j / 2 + 2].x, acc2[j / 2 + 2].y);
+          __nv_bfloat162 h3 = __floats2bfloat162_rn(acc2[j / 2 + 3].x, acc2[j / 2 + 3].y);
           v.x = *reinterpret_cast<uint32_t*>(&h0);
           v.y = *reinterpret_cast<uint32_t*>(&h1);
           v.z = *reinterpret_cast<uint32_t*>(&h2);

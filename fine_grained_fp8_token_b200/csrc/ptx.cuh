@@ -189,6 +189,15 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
       : "r"(taddr));
 }
 
+// COLS (32 or 64) consecutive fp32 columns of this thread's TMEM lane:
+// one or two 32x32b.x32 loads (complete after tmem_wait_ld).
+template <int COLS>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[COLS]) {
+  static_assert(COLS == 32 || COLS == 64, "32 or 64 columns");
+  tmem_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+  if constexpr (COLS == 64) tmem_ld_32x32b_x32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+}
+
 // ------------------------------------------------------------ block-scaled MMA (UE8M0)
 // D[tmem] (+)= (A * 2^(sfa-127)) x (B * 2^(sfb-127))^T with one UE8M0 scale
 // per row and 32-element K slice (kind::mxf8f6f4.block_scale, scale_vec 1X),
