@@ -159,12 +159,16 @@ fgfp8_status launch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const 
                          void* Y, int64_t M, int64_t N, int64_t K, const int32_t* offs, int E, int64_t b_rows,
                          cudaStream_t stream, int dev, int sm_count, int early) {
   using C = fgfp8::GemmCfg<BN, CW>;
-  CUtensorMap mA, mB;
+  CUtensorMap mA, mB, mBh;
   fgfp8_status st = make_map_u8_sw128(&mA, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
                                       static_cast<uint64_t>(K), 128);
   if (st != FGFP8_OK) return st;
   st = make_map_u8_sw128(&mB, Wq, static_cast<uint64_t>(b_rows), static_cast<uint64_t>(K), static_cast<uint64_t>(K),
                          BN);
+  if (st != FGFP8_OK) return st;
+  // the same weights with a 128-row box, for half tiles
+  st = make_map_u8_sw128(&mBh, Wq, static_cast<uint64_t>(b_rows), static_cast<uint64_t>(K), static_cast<uint64_t>(K),
+                         BN / 2);
   if (st != FGFP8_OK) return st;
   auto kernel = fgfp8::gemm_blockscaled_kernel<BN, CW, FMT, kGrouped>;
   st = set_smem(reinterpret_cast<const void*>(kernel), C::kSmemBytes, dev);
@@ -184,10 +188,21 @@ fgfp8_status launch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const 
   const int64_t tiles = ((M + C::kBM - 1) / C::kBM) * (N / BN);
   if (tiles == 0) return ok();
   const int64_t grid = tiles < sm_count ? tiles : sm_count;
+  // Dense 256-wide tiles: when the last partial wave of R full tiles fits
+  // twice into one wave (2R <= grid), those R tiles run as 2R half tiles,
+  // so that wave takes about half a tile's time instead of a whole one.
+  int64_t num_full = tiles, items = tiles;
+  if (!kGrouped && BN == 256) {
+    const int64_t waves = tiles / grid, rest = tiles - waves * grid;
+    if (waves >= 1 && rest > 0 && 2 * rest <= grid) {
+      num_full = waves * grid;
+      items = num_full + 2 * rest;
+    }
+  }
   return launch_dependent(kernel, static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, stream, "gemm launch", mA,
-                          mB, Xs, static_cast<uint32_t>(ld_s), Ws, reinterpret_cast<__nv_bfloat16*>(Y),
+                          mB, mBh, Xs, static_cast<uint32_t>(ld_s), Ws, reinterpret_cast<__nv_bfloat16*>(Y),
                           static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), offs, E,
-                          static_cast<int>(tiles), early);
+                          static_cast<int>(items), static_cast<int>(num_full), early);
 }
 
 // UE8M0 launch with hardware block scaling (persistent, 128 x BN tiles).

@@ -31,6 +31,7 @@
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
+#include <type_traits>
 
 #include "ptx.cuh"
 
@@ -105,7 +106,7 @@ __device__ __forceinline__ float combine_raw(uint32_t a, uint32_t w) {
 }
 
 // Depth (in K blocks) of the scale prefetch ring of the promotion warps.
-constexpr int kScaleAhead = 4;
+constexpr int kScaleAhead = 2;
 
 // Expert owning row m: the e with offs[e] <= m < offs[e+1] (binary search),
 // or -1 when the offsets are inconsistent with m.
@@ -198,13 +199,21 @@ __device__ __forceinline__ void issue_mmas(uint32_t a_base, uint32_t b_base, int
   if (!mbar_wait(mma_done, 0)) record_status(kDevTimeoutMma);
 }
 
+// Dense 128 x 256 tiles may end with half tiles: work items t >= num_full
+// split the remaining full tiles f = num_full + (t - num_full) / 2 into two
+// 128 x 128 halves, loaded through tmBh (a 128-row box of the same weights)
+// and promoted by all promotion warps at CW/2 columns each.  The host uses
+// them when the last partial wave of full tiles fits twice into one wave, so
+// that wave takes about half as long.
 template <int BN, int CW, int FMT, bool kGrouped>
 __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
     gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                            const void* __restrict__ Xs, uint32_t ld_s, const void* __restrict__ Ws,
-                            __nv_bfloat16* __restrict__ Y, int M, int N, int K,
-                            const int32_t* __restrict__ group_offs, int E, int num_tiles, int early_b) {
+                            const __grid_constant__ CUtensorMap tmBh, const void* __restrict__ Xs, uint32_t ld_s,
+                            const void* __restrict__ Ws, __nv_bfloat16* __restrict__ Y, int M, int N, int K,
+                            const int32_t* __restrict__ group_offs, int E, int num_tiles, int num_full,
+                            int early_b) {
   using C = GemmCfg<BN, CW>;
+  constexpr bool kHalfTiles = !kGrouped && BN == 256;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -224,15 +233,22 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
   const int num_m = (M + C::kBM - 1) / C::kBM;
   const int num_n = N / BN;
 
-  // Tile t -> (m0, n0, expert).  Dense tiles run M-fastest (the activation
-  // tile set stays L2-resident while a weight tile is reused); grouped tiles
-  // run N-fastest (the CTAs of one expert share its weights in L2).  An
-  // expert of -1 marks a tile whose rows no segment covers: every role skips
-  // it and the status word records it.
-  auto coords = [&](int t, int& m0, int& n0, int& expert) {
+  // Work item t -> (m0, n0, expert, half).  Dense tiles run M-fastest (the
+  // activation tile set stays L2-resident while a weight tile is reused);
+  // grouped tiles run N-fastest (the CTAs of one expert share its weights in
+  // L2).  An expert of -1 marks a tile whose rows no segment covers: every
+  // role skips it and the status word records it.
+  auto coords = [&](int t, int& m0, int& n0, int& expert, bool& half) {
+    half = false;
     if (!kGrouped) {
-      m0 = (t % num_m) * C::kBM;
-      n0 = (t / num_m) * BN;
+      int f = t, h = 0;
+      if (kHalfTiles && t >= num_full) {
+        f = num_full + ((t - num_full) >> 1);
+        h = (t - num_full) & 1;
+        half = true;
+      }
+      m0 = (f % num_m) * C::kBM;
+      n0 = (f / num_m) * BN + h * (BN / 2);
       expert = 0;
     } else {
       n0 = (t % num_n) * BN;
@@ -256,6 +272,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (kHalfTiles) tma_prefetch_desc(&tmBh);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::kTmemCols);
@@ -277,9 +294,11 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
       // blocks are requested before the wait (the weights must not be
       // written by the preceding grid).
       int pre = 0;
-      if (!kGrouped && early_b && static_cast<int>(blockIdx.x) < num_tiles) {
-        int m0, n0, expert;
-        coords(blockIdx.x, m0, n0, expert);
+      bool half0 = true;
+      int m0p = 0, n0p = 0, ep = 0;
+      if (static_cast<int>(blockIdx.x) < num_tiles) coords(blockIdx.x, m0p, n0p, ep, half0);
+      if (!kGrouped && early_b && static_cast<int>(blockIdx.x) < num_tiles && !half0) {
+        const int n0 = n0p;
         pre = KB < C::kStages ? KB : C::kStages;
         for (int kb = 0; kb < pre; ++kb) {
           mbar_arrive_expect_tx(&full[kb], C::kStageBytes);
@@ -291,12 +310,15 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         int m0, n0, expert;
-        coords(t, m0, n0, expert);
+        bool half;
+        coords(t, m0, n0, expert, half);
         if (expert < 0) {
           record_status(kDevBadGroupOffsets);
           continue;
         }
         const int b_row = expert * N + n0;
+        const CUtensorMap* mapB = (kHalfTiles && half) ? &tmBh : &tmB;
+        const uint32_t stage_tx = (kHalfTiles && half) ? C::kABytes + C::kBBytes / 2 : C::kStageBytes;
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % C::kStages;
           if (it >= static_cast<uint32_t>(C::kStages) && !mbar_wait(&empty[s], ((it / C::kStages) & 1u) ^ 1u)) {
@@ -305,8 +327,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
             break;
           }
           if (it >= static_cast<uint32_t>(pre)) {
-            mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-            tma_load_2d(sB + s * C::kBBytes, &tmB, &full[s], kb * C::kBK, b_row);
+            mbar_arrive_expect_tx(&full[s], stage_tx);
+            tma_load_2d(sB + s * C::kBBytes, mapB, &full[s], kb * C::kBK, b_row);
           }
           tma_load_2d(sA + s * C::kABytes, &tmA, &full[s], kb * C::kBK, m0);
         }
@@ -316,7 +338,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
         if (!mbar_wait(&full[j % C::kStages], (j / C::kStages) & 1u)) record_status(kDevTimeoutProducer);
     } else if (warp == 1 && lane == 0) {
       // ================= MMA issuer
-      constexpr uint32_t idesc = idesc_e4m3_f32(128, BN);
+      constexpr uint32_t idesc_full = idesc_e4m3_f32(128, BN);
+      constexpr uint32_t idesc_half = idesc_e4m3_f32(128, BN / 2);
       const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
       // descriptors differ per stage / K step only in the start-address field
       const uint64_t a_desc0 = smem_desc_k_sw128(a_base), b_desc0 = smem_desc_k_sw128(b_base);
@@ -324,8 +347,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         int m0, n0, expert;
-        coords(t, m0, n0, expert);
+        bool half;
+        coords(t, m0, n0, expert, half);
         if (expert < 0) continue;
+        const uint32_t idesc = (kHalfTiles && half) ? idesc_half : idesc_full;
         for (int kb = 0; kb < KB; ++kb, ++it, ++bt) {
           const int s = it % C::kStages;
           const int buf = bt % C::kNumBuf;
@@ -360,10 +385,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
     // ================= promotion / epilogue
     const int ew = warp - 4;
     const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
-    const int grp = ew >> 2;                   // column group: columns [grp * CW, grp * CW + CW)
-    const int col0 = grp * CW;
+    const int grp = ew >> 2;                   // column group: columns [grp * cols, grp * cols + cols)
     const int row = quad * 32 + lane;
-    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(col0);
     // raw scale words for K blocks kb .. kb+kScaleAhead-1, ring slot kb % kScaleAhead
     uint32_t ra[kScaleAhead], rw[kScaleAhead];
     auto fetch = [&](int kb, int m, bool live, uint64_t ws_row, uint32_t& a, uint32_t& w) {
@@ -375,9 +398,14 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
         w = 0u;
       }
     };
-    // this thread's row, liveness and weight-scale row in tile t (expert < 0: skipped tile)
-    auto tile_rows = [&](int t, int& m0, int& n0, int& expert, int& m, bool& live, uint64_t& ws_row) {
-      coords(t, m0, n0, expert);
+    // This thread's row, first column, liveness and weight-scale row in work
+    // item t (expert < 0: skipped tile).  A warp covers CW columns of a full
+    // tile, CW/2 of a half tile; either way they lie in one 128-column
+    // weight block.
+    auto tile_rows = [&](int t, int& m0, int& n0, int& expert, bool& half, int& col0, int& m, bool& live,
+                         uint64_t& ws_row) {
+      coords(t, m0, n0, expert, half);
+      col0 = grp * ((kHalfTiles && half) ? CW / 2 : CW);
       m = m0 + row;
       live = (m < M) && (n0 + col0 < N);
       ws_row = (static_cast<uint64_t>(expert < 0 ? 0 : expert) * NB + (n0 + col0) / 128) * KB;
@@ -385,21 +413,17 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
     int pref_t = -1;                           // tile whose first scale words are in the ring
     uint32_t bt = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-      int m0, n0, expert, m;
-      bool live;
-      uint64_t ws_row;
-      tile_rows(t, m0, n0, expert, m, live, ws_row);
-      if (expert < 0) continue;
-      if (pref_t != t) {
-#pragma unroll
-        for (int d = 0; d < kScaleAhead; ++d) fetch(d, m, live, ws_row, ra[d], rw[d]);
-      }
 
+    // One work item with COLS columns per warp: per K block, the partial from
+    // TMEM times sa * sw into the accumulators, then the bf16 epilogue.
+    auto promote = [&](auto cols_tag, int t, int m0, int n0, int col0, int m, bool live, uint64_t ws_row) {
+      constexpr int COLS = decltype(cols_tag)::value;
+      const uint32_t lane_base =
+          tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(col0);
       // fp32 accumulators as pairs: columns 2j, 2j+1 in acc2[j]
-      float2 acc2[CW / 2];
+      float2 acc2[COLS / 2];
 #pragma unroll
-      for (int j = 0; j < CW / 2; ++j) acc2[j] = make_float2(0.0f, 0.0f);
+      for (int j = 0; j < COLS / 2; ++j) acc2[j] = make_float2(0.0f, 0.0f);
       for (int kb0 = 0; kb0 < KB && ok; kb0 += kScaleAhead) {
 #pragma unroll
         for (int d = 0; d < kScaleAhead; ++d) {
@@ -416,11 +440,11 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
           }
           tc_fence_after();
           const uint32_t taddr = lane_base + static_cast<uint32_t>(buf * BN);
-          // Two halves of CW/2 columns, each one TMEM load round trip and
+          // Two halves of COLS/2 columns, each one TMEM load round trip and
           // packed fp32x2 FMAs (fma.rn per element, as a scalar FMA).  The
-          // buffer is handed back as soon as the second half is in registers;
-          // that half's FMAs run while the next MMA fills the buffer.
-          constexpr int kHalf = CW / 2;
+          // buffer is handed back as soon as the second half is in
+          // registers; that half's FMAs run while the next MMA fills it.
+          constexpr int kHalf = COLS / 2;
           const float2 sc2 = make_float2(sc, sc);
           uint32_t p[kHalf];
           tmem_ld_cols<kHalf>(taddr, p);
@@ -440,16 +464,16 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
           ++bt;
         }
       }
-      if (!ok) break;
+      if (!ok) return;
 
       // The next tile's first scale words: their latency overlaps the epilogue.
       pref_t = -1;
       if (t + static_cast<int>(gridDim.x) < num_tiles) {
         const int tn = t + static_cast<int>(gridDim.x);
-        int m0n, n0n, en, mn;
-        bool liven;
+        int m0n, n0n, en, c0n, mn;
+        bool hn, liven;
         uint64_t wsn;
-        tile_rows(tn, m0n, n0n, en, mn, liven, wsn);
+        tile_rows(tn, m0n, n0n, en, hn, c0n, mn, liven, wsn);
         if (en >= 0) {
 #pragma unroll
           for (int d = 0; d < kScaleAhead; ++d) fetch(d, mn, liven, wsn, ra[d], rw[d]);
@@ -464,7 +488,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
       // then reads back row 4i + l / 8, chunk l % 8, for i = 0..7.
       uint8_t* slot = sStg + ew * C::kWarpStageBytes;
 #pragma unroll
-      for (int p = 0; p < CW / 64; ++p) {
+      for (int p = 0; p < COLS / 64; ++p) {
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           const int j = p * 64 + c * 8;
@@ -489,6 +513,25 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
         }
         __syncwarp();
       }
+    };
+
+    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      int m0, n0, expert, col0, m;
+      bool half, live;
+      uint64_t ws_row;
+      tile_rows(t, m0, n0, expert, half, col0, m, live, ws_row);
+      if (expert < 0) continue;
+      if (pref_t != t) {
+#pragma unroll
+        for (int d = 0; d < kScaleAhead; ++d) fetch(d, m, live, ws_row, ra[d], rw[d]);
+      }
+      if constexpr (kHalfTiles) {
+        if (half) {
+          promote(std::integral_constant<int, CW / 2>{}, t, m0, n0, col0, m, live, ws_row);
+          continue;
+        }
+      }
+      promote(std::integral_constant<int, CW>{}, t, m0, n0, col0, m, live, ws_row);
     }
   }
 

@@ -83,6 +83,19 @@ def test_gemm_zero_and_unit_codes(dev):
     assert (Y.float() == 0).all()
 
 
+@pytest.mark.parametrize("M,N,K", [(1200, 4096, 256), (2560, 2304, 384)])
+def test_gemm_half_tile_tail(dev, M, N, K):
+    """Shapes whose last partial wave of 128x256 tiles runs as 128x128 half
+    tiles on a 148-SM B200 (1200x4096: 160 tiles = 148 + 12, ragged last
+    M tile; 2560x2304: 180 tiles = 148 + 32): every output against the
+    oracle."""
+    cfg = workloads.scaled_linear(workloads.TINY, M=M, N=N, K=K, seed=M + N + K)
+    X, W = workloads.linear_inputs(cfg)
+    Y = gpu_linear(X.to(dev), W.to(dev), F32)
+    Y_ref, S = oracle_linear(bits16(X), bits16(W), F32)
+    assert_gemm_close(y_to_f64(Y), Y_ref, S, f"half-tile tail {M}x{N}x{K}")
+
+
 def sample_rows(M, n_random=48, seed=0):
     rng = np.random.default_rng(seed)
     tiles = np.arange(0, M, 128)
