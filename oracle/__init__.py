@@ -14,6 +14,9 @@ Sources (page title, section):
     per-token activation groups matching the weight's input-channel block (128).
   * "Fine-grained FP8", "DeepGEMM fast path": the dynamic activation scheme.
   * "Fine-grained FP8", "UE8M0 scale format": float8_e8m0fnu scales.
+  * "FP8 W8A8", "Applying quantization": the FP8_DYNAMIC scheme (per-channel
+    weights, per-token activations); the OwLite FP8 page: AbsMax per-tensor
+    scales (static activation scales).
 """
 from __future__ import annotations
 
@@ -82,6 +85,14 @@ def _load():
             lib.orc_grouped_gemm.argtypes = [P, P, i64, P, P, P, c.c_int32, i64, i64,
                                              c.c_int, P, i64, P, P, P]
             lib.orc_grouped_gemm.restype = c.c_int
+            lib.orc_quant_rows.argtypes = [P, i64, i64, i64, P, P]
+            lib.orc_quant_rows.restype = None
+            lib.orc_tensor_scale.argtypes = [P, i64, i64, i64]
+            lib.orc_tensor_scale.restype = c.c_float
+            lib.orc_quant_static.argtypes = [P, i64, i64, i64, c.c_float, P]
+            lib.orc_quant_static.restype = None
+            lib.orc_gemm_rowcol.argtypes = [P, P, c.c_int, P, P, c.c_int, i64, i64, P, i64, P, P]
+            lib.orc_gemm_rowcol.restype = None
             lib.orc_bf16_rne.argtypes = [c.c_double]
             lib.orc_bf16_rne.restype = c.c_uint16
             for name in ("orc_e4m3_encode_array", "orc_scale_f32_array",
@@ -270,6 +281,58 @@ def grouped_gemm(Xq, Xs, Wq, Ws, group_offs, fmt: int, rows=None):
                               _ptr(Y), _ptr(S), _ptr(scratch))
     if rc != 0:
         raise ValueError("a requested row lies outside every expert segment")
+    return Y, S
+
+
+# ---------------------------------------------------------------- row / tensor scales
+def quant_rows(X):
+    """One fp32 scale per row over all K ("FP8 W8A8", FP8_DYNAMIC: per-token
+    activations, per-output-channel weights).  X: bf16 [R, K].  Returns
+    (Xq u8 [R, K], scales fp32 [R])."""
+    lib = _load()
+    X = _u16(X)
+    R, K = X.shape
+    Xq = np.empty((R, K), dtype=np.uint8)
+    sc = np.empty(R, dtype=np.float32)
+    lib.orc_quant_rows(_ptr(X), R, K, K, _ptr(Xq), _ptr(sc))
+    return Xq, sc
+
+
+def tensor_scale(X) -> np.float32:
+    """Per-tensor AbsMax scale: max(amax(X), 1e-4) / 448 in fp32."""
+    lib = _load()
+    X = _u16(X)
+    R, K = X.shape
+    return np.float32(lib.orc_tensor_scale(_ptr(X), R, K, K))
+
+
+def quant_static(X, scale) -> np.ndarray:
+    """Codes of X / scale for a given (static) fp32 scale."""
+    lib = _load()
+    X = _u16(X)
+    R, K = X.shape
+    Xq = np.empty((R, K), dtype=np.uint8)
+    lib.orc_quant_static(_ptr(X), R, K, K, float(np.float32(scale)), _ptr(Xq))
+    return Xq
+
+
+def gemm_rowcol(Xq, sx, Wq, sw, rows=None):
+    """Row/column-scaled GEMM reference: Y[m, n] = sx[m] * sw[n] *
+    sum_k x_code * w_code, with a one-element sx or sw meaning a per-tensor
+    scale.  Returns (Y fp64 [R, N], S fp64 [R, N])."""
+    lib = _load()
+    Xq = np.ascontiguousarray(Xq)
+    Wq = np.ascontiguousarray(Wq)
+    sx = np.ascontiguousarray(sx, dtype=np.float32).reshape(-1)
+    sw = np.ascontiguousarray(sw, dtype=np.float32).reshape(-1)
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    assert sx.size in (1, M) and sw.size in (1, N)
+    rows = np.arange(M, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    Y = np.empty((len(rows), N), dtype=np.float64)
+    S = np.empty((len(rows), N), dtype=np.float64)
+    lib.orc_gemm_rowcol(_ptr(Xq), _ptr(sx), int(sx.size == 1 and M != 1), _ptr(Wq), _ptr(sw),
+                        int(sw.size == 1 and N != 1), N, K, _ptr(rows), len(rows), _ptr(Y), _ptr(S))
     return Y, S
 
 

@@ -322,6 +322,72 @@ int orc_grouped_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s,
     return 0;
 }
 
+/* ------------------------------------------------------------------ */
+/* Row and tensor scale granularity ("FP8 W8A8", "Applying quantization": */
+/* the FP8_DYNAMIC scheme quantizes weights statically per output channel */
+/* and activations dynamically per token; "Fine-grained FP8", "DeepGEMM   */
+/* fast path", and the OwLite FP8 page's AbsMax per-tensor calibration:    */
+/* static per-tensor scales).  Same scale and code rules as above, with   */
+/* the group widened to a whole row of K, or to the whole tensor.         */
+/* ------------------------------------------------------------------ */
+
+/* One fp32 scale per row r of X [R, K]: s[r] = max(amax(row), 1e-4) / 448,
+ * codes Xq[r, k] = e4m3(X[r, k] / s[r]). */
+void orc_quant_rows(const uint16_t* X, int64_t R, int64_t K, int64_t ldx,
+                    uint8_t* Xq, float* scales) {
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; ++r) {
+        const uint16_t* xr = X + r * ldx;
+        float s = orc_scale_f32(amax_clamped(xr, K, 0, 1));
+        scales[r] = s;
+        quantize_run(xr, K, s, Xq + r * K);
+    }
+}
+
+/* Per-tensor scale: max(amax over all R x K elements, 1e-4) / 448. */
+float orc_tensor_scale(const uint16_t* X, int64_t R, int64_t K, int64_t ldx) {
+    return orc_scale_f32(amax_clamped(X, K, ldx, R));
+}
+
+/* Static quantization with a given scale s: Xq = e4m3(X / s). */
+void orc_quant_static(const uint16_t* X, int64_t R, int64_t K, int64_t ldx,
+                      float s, uint8_t* Xq) {
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; ++r) quantize_run(X + r * ldx, K, s, Xq + r * K);
+}
+
+/* Row/column-scaled GEMM:
+ *   Y[m,n] = sx[m] * sw[n] * sum_k e4m3(Xq[m,k]) * e4m3(Wq[n,k])
+ * with sx[0] for every m when x_per_tensor, sw[0] for every n when
+ * w_per_tensor.  The K sum is exact in fp64 for K < 2^17 (each product is a
+ * multiple of 2^-18 below 2^18).  S[m,n] = sum_k |x_hat * w_hat|.  rows as
+ * in orc_gemm. */
+void orc_gemm_rowcol(const uint8_t* Xq, const float* sx, int x_per_tensor,
+                     const uint8_t* Wq, const float* sw, int w_per_tensor,
+                     int64_t N, int64_t K, const int64_t* rows, int64_t nrows,
+                     double* Y, double* S) {
+    double table[256];
+    for (int c = 0; c < 256; ++c) table[c] = orc_e4m3_decode((uint8_t)c);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t m = rows[r];
+        const uint8_t* xr = Xq + m * K;
+        double a = (double)sx[x_per_tensor ? 0 : m];
+        for (int64_t n = 0; n < N; ++n) {
+            const uint8_t* wr = Wq + n * K;
+            double p = 0.0, pabs = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double prod = table[xr[k]] * table[wr[k]];
+                p += prod;
+                pabs += fabs(prod);
+            }
+            double c = a * (double)sw[w_per_tensor ? 0 : n];
+            Y[r * N + n] = c * p;
+            S[r * N + n] = fabs(c) * pabs;
+        }
+    }
+}
+
 /* bf16 round-to-nearest-even of an fp64 value, for reporting only. */
 uint16_t orc_bf16_rne(double v) {
     if (isnan(v)) return 0x7FC0;

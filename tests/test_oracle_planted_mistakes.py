@@ -15,7 +15,8 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "oracle.c")
-PIN_TESTS = ["tests/test_oracle_codec.py", "tests/test_oracle_quant.py", "tests/test_oracle_gemm.py"]
+PIN_TESTS = ["tests/test_oracle_codec.py", "tests/test_oracle_quant.py", "tests/test_oracle_gemm.py",
+             "tests/test_oracle_rowcol.py"]
 
 MUTANTS = {
     "tie_to_odd": ("pick = (lo % 2 == 0) ? lo : up;", "pick = (lo % 2 == 0) ? up : lo;"),
@@ -40,6 +41,16 @@ MUTANTS = {
                         "double prod = table[xr[k]] * fabs(table[wr[k]]);"),
     "grouped_segment_boundary": ("if (offs[i] <= m && m < offs[i + 1]) { e = i; break; }",
                                  "if (offs[i] <= m && m <= offs[i + 1]) { e = i; break; }"),
+    "row_amax_half_row": ("float s = orc_scale_f32(amax_clamped(xr, K, 0, 1));",
+                          "float s = orc_scale_f32(amax_clamped(xr, K / 2, 0, 1));"),
+    "tensor_amax_first_row": ("return orc_scale_f32(amax_clamped(X, K, ldx, R));",
+                              "return orc_scale_f32(amax_clamped(X, K, ldx, 1));"),
+    "static_multiplies_by_scale": ("for (int64_t r = 0; r < R; ++r) quantize_run(X + r * ldx, K, s, Xq + r * K);",
+                                   "for (int64_t r = 0; r < R; ++r) quantize_run(X + r * ldx, K, 1.0f / s, Xq + r * K);"),
+    "rowcol_channel_scale_ignored": ("double c = a * (double)sw[w_per_tensor ? 0 : n];",
+                                     "double c = a * (double)sw[0];"),
+    "rowcol_token_scale_indexed_by_n": ("double a = (double)sx[x_per_tensor ? 0 : m];",
+                                        "double a = (double)sx[x_per_tensor ? 0 : (m % 2)];"),
 }
 
 
