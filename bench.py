@@ -12,7 +12,10 @@ pre-quantized weights.
 
 Default workload: the Llama-3-8B attention projection in prefill,
 X [4096, 4096] x W [4096, 4096], fp32 block scales.  Other workloads can be
-chosen with --workload (see workloads/).
+chosen with --workload (see workloads/), among them the same dense shapes
+with per-token x per-channel scales (the FP8_DYNAMIC scheme) or a static
+per-tensor activation scale, whose step is the row / tensor quantizer and
+the row/column-scaled GEMM.
 
 Timing: W warm-up steps, then K timed steps.  L2 is flushed (a 256 MB write followed
 by a 256 MB read, so no dirty line is written back inside the next step)
@@ -49,11 +52,23 @@ L2_FLUSH_BYTES = 256 << 20
 FP8_OVER_BF16 = 2.0            # nominal dense fp8 / bf16 tensor ratio on B200 (4.5 / 2.25 PFLOP/s)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
+# Row / tensor scale granularity on the dense shapes ("FP8 W8A8", "Applying
+# quantization"): "fp8_dynamic" = per-token activations x per-output-channel
+# weights; "static_tensor" = one static activation scale (AbsMax over the
+# layer's input, calibrated once before timing) x per-channel weights.
+ROWCOL_SCHEMES = ("fp8_dynamic", "static_tensor")
+ROWCOL = {f"{c.name}_{sch}": (c, sch) for c in (workloads.LLAMA_ATTN, workloads.LLAMA_GATE_UP, workloads.LLAMA_DOWN)
+          for sch in ROWCOL_SCHEMES}
+
 WORKLOAD_ALIASES = {
     "llama_attn": workloads.LLAMA_ATTN.name, "tiny": workloads.TINY.name,
     "llama_gate_up": workloads.LLAMA_GATE_UP.name, "llama_down": workloads.LLAMA_DOWN.name,
     **{f"ds_decode_m{m}": workloads.DS_DECODE[m].name for m in (1, 8, 32, 64)},
     "moe": workloads.MOE.name, "moe_small": workloads.MOE_SMALL.name,
+    "llama_attn_dynamic": f"{workloads.LLAMA_ATTN.name}_fp8_dynamic",
+    "llama_attn_static": f"{workloads.LLAMA_ATTN.name}_static_tensor",
+    "llama_gate_up_dynamic": f"{workloads.LLAMA_GATE_UP.name}_fp8_dynamic",
+    "llama_down_dynamic": f"{workloads.LLAMA_DOWN.name}_fp8_dynamic",
 }
 
 
@@ -231,6 +246,75 @@ class DenseLayer:
         return "gemm_blockscaled_kernel" if self.cfg.fmt == 0 else "gemm_mx_kernel"
 
 
+class RowColLayer:
+    """One dense layer with row / tensor scale granularity: per-output-channel
+    weight scales (fgfp8_quant_rows on W) and either per-token activation
+    scales (fgfp8_quant_rows on X, the FP8_DYNAMIC scheme) or one static
+    activation scale calibrated once from the layer's input
+    (fgfp8_tensor_scale, then fgfp8_quant_static per step).  The GEMM is
+    fgfp8_gemm_rowcol."""
+
+    def __init__(self, cfg: workloads.Linear, scheme: str, dev):
+        import fine_grained_fp8_token_b200 as fg
+        self.fg, self.cfg, self.scheme, self.dev = fg, cfg, scheme, dev
+        self.X = workloads.activations((cfg.M, cfg.K), cfg.x_kind, cfg.seed, device=dev)
+        self.W = workloads.weights((cfg.N, cfg.K), cfg.seed + 1, device=dev)
+        self.Wq = torch.empty((cfg.N, cfg.K), dtype=torch.uint8, device=dev)
+        self.sw = torch.empty((cfg.N,), dtype=torch.float32, device=dev)
+        self.Xq = torch.empty((cfg.M, cfg.K), dtype=torch.uint8, device=dev)
+        if scheme == "fp8_dynamic":
+            self.sx = torch.empty((cfg.M,), dtype=torch.float32, device=dev)
+        else:
+            self.sx = fg.tensor_scale(self.X)             # calibration, before timing
+        self.Y = torch.empty((cfg.M, cfg.N), dtype=torch.bfloat16, device=dev)
+        self.quant_weight()
+
+    def quant_weight(self):
+        self.fg.quant_rows(self.W, Xq=self.Wq, scales=self.sw)
+
+    def quant_act(self, X=None):
+        X = self.X if X is None else X
+        if self.scheme == "fp8_dynamic":
+            self.fg.quant_rows(X, Xq=self.Xq, scales=self.sx)
+        else:
+            self.fg.quant_static(X, self.sx, Xq=self.Xq)
+
+    def gemm(self):
+        self.fg.gemm_rowcol(self.Xq, self.sx, self.Wq, self.sw, Y=self.Y)
+
+    def linear(self, X=None):
+        self.quant_act(X)
+        self.gemm()
+
+    def flops(self):
+        c = self.cfg
+        return 2.0 * c.M * c.N * c.K
+
+    def act_bytes(self):
+        c = self.cfg
+        return 3.0 * c.M * c.K + (4.0 * c.M if self.scheme == "fp8_dynamic" else 0.0)
+
+    def gemm_bytes(self):
+        c = self.cfg
+        return c.M * c.K + c.N * c.K + 4.0 * (c.M + c.N) + 2.0 * c.M * c.N
+
+    def weight_bytes(self):
+        c = self.cfg
+        return 3.0 * c.N * c.K + 4.0 * c.N
+
+    def describe(self):
+        c = self.cfg
+        x = "per-token (dynamic)" if self.scheme == "fp8_dynamic" else "per-tensor (static, calibrated once)"
+        return {"workload": f"{c.name}_{self.scheme}", "M": c.M, "N": c.N, "K": c.K,
+                "scales": f"fp32, activations {x}, weights per output channel", "x": c.x_kind}
+
+    def host_io(self):
+        return self.X, self.Y
+
+    def gemm_kernel_name(self):
+        return "gemm_rowcol_kernel"
+
+
 class MoELayer:
     """Grouped expert layer: routed token rows and pre-quantized experts."""
 
@@ -299,6 +383,9 @@ class MoELayer:
 
 def make_layer(name, dev):
     name = WORKLOAD_ALIASES.get(name, name)
+    if name in ROWCOL:
+        cfg, scheme = ROWCOL[name]
+        return RowColLayer(cfg, scheme, dev)
     for cfg in (workloads.MOE, workloads.MOE_SMALL):
         if name == cfg.name:
             return MoELayer(cfg, dev)
@@ -436,6 +523,19 @@ class OracleSample:
         import oracle
         self.oracle = oracle
         name = WORKLOAD_ALIASES.get(name, name)
+        self.scheme = None
+        if name in ROWCOL:
+            cfg, self.scheme = ROWCOL[name]
+            X, W = workloads.linear_inputs(cfg)
+            self.N, self.K, self.fmt = cfg.N, cfg.K, cfg.fmt
+            xb = X.contiguous().view(torch.int16).numpy().view(np.uint16)
+            self.sx_static = oracle.tensor_scale(xb) if self.scheme == "static_tensor" else None
+            self.X = np.ascontiguousarray(xb[:rows])
+            self.Wq, self.sw = oracle.quant_rows(W.contiguous().view(torch.int16).numpy().view(np.uint16))
+            self.rows = self.X.shape[0]
+            self.desc = (f"first {self.rows} of {cfg.M} rows x the full [{cfg.N}, {cfg.K}] weight, "
+                         f"{self.scheme} scales")
+            return
         if name in (workloads.MOE.name, workloads.MOE_SMALL.name):
             cfg = workloads.MOE if name == workloads.MOE.name else workloads.MOE_SMALL
             r = workloads.moe_routing(cfg)
@@ -456,6 +556,14 @@ class OracleSample:
         self.rows = self.X.shape[0]
 
     def step(self):
+        if self.scheme == "fp8_dynamic":
+            Xq, sx = self.oracle.quant_rows(self.X)
+            self.oracle.gemm_rowcol(Xq, sx, self.Wq, self.sw)
+            return
+        if self.scheme == "static_tensor":
+            Xq = self.oracle.quant_static(self.X, self.sx_static)
+            self.oracle.gemm_rowcol(Xq, np.array([self.sx_static], dtype=np.float32), self.Wq, self.sw)
+            return
         Xq, Xs = self.oracle.quant_act(self.X, self.fmt)
         self.oracle.gemm(Xq, Xs, self.Wq, self.Ws, self.fmt)
 
@@ -591,7 +699,10 @@ def main():
                                      "bytes": layer.weight_bytes()},
             "apart_sum_us": 1e3 * (r["quant_ms"] + r["gemm_ms"]),
         },
-        "step_call": "fgfp8_grouped_linear" if isinstance(layer, MoELayer) else "fgfp8_linear",
+        "step_call": ("fgfp8_grouped_linear" if isinstance(layer, MoELayer) else
+                      ("fgfp8_quant_rows + fgfp8_gemm_rowcol" if getattr(layer, "scheme", None) == "fp8_dynamic"
+                       else "fgfp8_quant_static + fgfp8_gemm_rowcol") if isinstance(layer, RowColLayer)
+                      else "fgfp8_linear"),
         "e2e": {"value": whole_job_rate(world, flops, r["e2e_ms"]), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"], "ms_per_step": r["e2e_ms"]},
         "gpu_launches": r["launches"],

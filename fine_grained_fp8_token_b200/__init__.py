@@ -37,6 +37,10 @@ SIGNATURES = {
     "fgfp8_linear": (_INT, [_P, _I64, _P, _P, _I64, _P, _P, _P, _I64, _I64, _I64, _INT, _P]),
     "fgfp8_grouped_linear": (_INT, [_P, _I64, _P, _P, _I64, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _INT, _P]),
     "fgfp8_linear_noalloc": (_INT, [_P, _I64, _P, _P, _P, _I64, _I64, _I64, _INT, _P]),
+    "fgfp8_quant_rows": (_INT, [_P, _I64, _I64, _I64, _P, _P, _P]),
+    "fgfp8_tensor_scale": (_INT, [_P, _I64, _I64, _I64, _P, _P]),
+    "fgfp8_quant_static": (_INT, [_P, _I64, _I64, _I64, _P, _P, _P]),
+    "fgfp8_gemm_rowcol": (_INT, [_P, _P, _INT, _P, _P, _INT, _P, _I64, _I64, _I64, _P]),
     "fgfp8_check_device_status": (_INT, [_P]),
 }
 
@@ -96,6 +100,10 @@ fgfp8_grouped_gemm = _raw("fgfp8_grouped_gemm")
 fgfp8_linear = _raw("fgfp8_linear")
 fgfp8_grouped_linear = _raw("fgfp8_grouped_linear")
 fgfp8_linear_noalloc = _raw("fgfp8_linear_noalloc")
+fgfp8_quant_rows = _raw("fgfp8_quant_rows")
+fgfp8_tensor_scale = _raw("fgfp8_tensor_scale")
+fgfp8_quant_static = _raw("fgfp8_quant_static")
+fgfp8_gemm_rowcol = _raw("fgfp8_gemm_rowcol")
 fgfp8_check_device_status = _raw("fgfp8_check_device_status")
 
 
@@ -215,6 +223,59 @@ def grouped_linear(X, Wq, Ws, group_offs, fmt: int, Y=None, Xq=None, Xs=None, ld
     _check(fgfp8_grouped_linear(X.data_ptr(), X.stride(0), Xq.data_ptr(), Xs.data_ptr(), ld_s, Wq.data_ptr(),
                                 Ws.data_ptr(), Y.data_ptr(), group_offs.data_ptr(), E, M_total, N, K, fmt,
                                 _stream(stream)), "fgfp8_grouped_linear")
+    return Y
+
+
+# ---------------------------------------------------------------- row / tensor scales
+def quant_rows(X, Xq=None, scales=None, stream=None):
+    """One fp32 scale per row of X (bf16 [R, K], CUDA): per-token
+    activations or per-output-channel weights.  Returns (Xq uint8 [R, K],
+    scales fp32 [R])."""
+    import torch
+    R, K = X.shape
+    if Xq is None:
+        Xq = torch.empty((R, K), dtype=torch.uint8, device=X.device)
+    if scales is None:
+        scales = torch.empty((R,), dtype=torch.float32, device=X.device)
+    _check(fgfp8_quant_rows(X.data_ptr(), R, K, X.stride(0), Xq.data_ptr(), scales.data_ptr(), _stream(stream)),
+           "fgfp8_quant_rows")
+    return Xq, scales
+
+
+def tensor_scale(X, scale=None, stream=None):
+    """Per-tensor AbsMax scale of X (bf16 [R, K], CUDA) as a float32 [1] tensor."""
+    import torch
+    R, K = X.shape
+    if scale is None:
+        scale = torch.empty((1,), dtype=torch.float32, device=X.device)
+    _check(fgfp8_tensor_scale(X.data_ptr(), R, K, X.stride(0), scale.data_ptr(), _stream(stream)),
+           "fgfp8_tensor_scale")
+    return scale
+
+
+def quant_static(X, scale, Xq=None, stream=None):
+    """Codes of X / scale for a given float32 [1] device scale.  Returns Xq."""
+    import torch
+    R, K = X.shape
+    if Xq is None:
+        Xq = torch.empty((R, K), dtype=torch.uint8, device=X.device)
+    _check(fgfp8_quant_static(X.data_ptr(), R, K, X.stride(0), scale.data_ptr(), Xq.data_ptr(), _stream(stream)),
+           "fgfp8_quant_static")
+    return Xq
+
+
+def gemm_rowcol(Xq, sx, Wq, sw, Y=None, stream=None):
+    """Y = sx[m] sw[n] sum_k Xq Wq (bf16 [M, N]); a one-element sx or sw is a
+    per-tensor scale."""
+    import torch
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=Xq.device)
+    x_t = int(sx.numel() == 1 and M != 1)
+    w_t = int(sw.numel() == 1 and N != 1)
+    _check(fgfp8_gemm_rowcol(Xq.data_ptr(), sx.data_ptr(), x_t, Wq.data_ptr(), sw.data_ptr(), w_t, Y.data_ptr(),
+                             M, N, K, _stream(stream)), "fgfp8_gemm_rowcol")
     return Y
 
 

@@ -281,6 +281,54 @@ fgfp8_status dispatch_decode(const uint8_t* Xq, const void* Xs, int64_t ld_s, co
   return launch_decode<64, FMT>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev, early);
 }
 
+// Row/column-scaled GEMM: persistent grid of 128 x BN tiles.
+template <int BN>
+fgfp8_status launch_gemm_rowcol(const uint8_t* Xq, const float* sx, int x_per_tensor, const uint8_t* Wq,
+                                const float* sw, int w_per_tensor, void* Y, int64_t M, int64_t N, int64_t K,
+                                cudaStream_t stream, int dev, int sm_count) {
+  using C = fgfp8::RowColCfg<BN>;
+  CUtensorMap mA, mB;
+  fgfp8_status st = make_map_u8_sw128(&mA, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
+                                      static_cast<uint64_t>(K), 128);
+  if (st != FGFP8_OK) return st;
+  st = make_map_u8_sw128(&mB, Wq, static_cast<uint64_t>(N), static_cast<uint64_t>(K), static_cast<uint64_t>(K), BN);
+  if (st != FGFP8_OK) return st;
+  auto kernel = fgfp8::gemm_rowcol_kernel<BN>;
+  st = set_smem(reinterpret_cast<const void*>(kernel), C::kSmemBytes, dev);
+  if (st != FGFP8_OK) return st;
+  const int64_t tiles = ((M + C::kBM - 1) / C::kBM) * (N / BN);
+  if (tiles == 0) return ok();
+  const int64_t grid = tiles < sm_count ? tiles : sm_count;
+  return launch_dependent(kernel, static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, stream,
+                          "row/column-scaled gemm launch", mA, mB, sx, x_per_tensor, sw, w_per_tensor,
+                          reinterpret_cast<__nv_bfloat16*>(Y), static_cast<int>(M), static_cast<int>(N),
+                          static_cast<int>(K), static_cast<int>(tiles));
+}
+
+// Shared checks of the row / tensor quantizers' input X bf16 [R, K] (row
+// stride ldx) and, when given, their codes Xq u8 [R, K].
+fgfp8_status check_rows_common(const void* X, int64_t R, int64_t K, int64_t ldx, bool has_codes,
+                               const uint8_t* Xq) {
+  if (R < 0 || K < 0 || ldx < 0) return fail(FGFP8_ERR_INVALID_ARG, "negative size");
+  if (K == 0 || K % 128 != 0) return fail(FGFP8_ERR_SHAPE, "K must be a positive multiple of 128");
+  if (ldx < K) return fail(FGFP8_ERR_SHAPE, "ldx must be >= K");
+  if (R >= (int64_t(1) << 31) || R * (K / 8) >= (int64_t(1) << 32))
+    return fail(FGFP8_ERR_SHAPE, "R must be < 2^31 and R*K/8 < 2^32");
+  if (R > 0 && !X) return fail(FGFP8_ERR_INVALID_ARG, "X is NULL");
+  if (!aligned(X, 16) || ldx % 8 != 0) return fail(FGFP8_ERR_ALIGN, "X must be 16-byte aligned with ldx % 8 == 0");
+  if (has_codes) {
+    if (R > 0 && !Xq) return fail(FGFP8_ERR_INVALID_ARG, "Xq is NULL");
+    if (!aligned(Xq, 16)) return fail(FGFP8_ERR_ALIGN, "Xq must be 16-byte aligned");
+  }
+  return FGFP8_OK;
+}
+
+unsigned grid_stride_blocks(int64_t work_items, int sm_count) {
+  const int64_t want = (work_items + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(sm_count) * 8;
+  return static_cast<unsigned>(want < 1 ? 1 : (want < cap ? want : cap));
+}
+
 fgfp8_status check_gemm_common(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
                                void* Y, int64_t M, int64_t N, int64_t K, int fmt) {
   fgfp8_status st = check_fmt(fmt);
@@ -541,6 +589,94 @@ fgfp8_status fgfp8_linear_noalloc(const void* X, int64_t ldx, const uint8_t* Wq,
   st = quant_act_impl(X, M, K, ldx, Xq, Xs, ld_s, fmt, stream, false);
   if (st != FGFP8_OK) return st;
   return gemm_impl(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, fmt, stream, 1, false);
+}
+
+fgfp8_status fgfp8_quant_rows(const void* X, int64_t R, int64_t K, int64_t ldx, uint8_t* Xq, float* scales,
+                              void* stream) {
+  fgfp8_status st = check_rows_common(X, R, K, ldx, true, Xq);
+  if (st != FGFP8_OK) return st;
+  if (R == 0) return ok();
+  if (!scales) return fail(FGFP8_ERR_INVALID_ARG, "scales is NULL");
+  if (!aligned(scales, 4)) return fail(FGFP8_ERR_ALIGN, "scales must be 4-byte aligned");
+  int dev;
+  DeviceInfo info;
+  st = current_device(&dev, &info);
+  if (st != FGFP8_OK) return st;
+  fgfp8::quant_rows_kernel<<<static_cast<unsigned>(R), fgfp8::kRowThreads, 0,
+                             reinterpret_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint16_t*>(X), static_cast<uint32_t>(K), static_cast<uint64_t>(ldx), Xq, scales);
+  return check_launch("quant_rows launch");
+}
+
+fgfp8_status fgfp8_tensor_scale(const void* X, int64_t R, int64_t K, int64_t ldx, float* scale, void* stream) {
+  fgfp8_status st = check_rows_common(X, R, K, ldx, false, nullptr);
+  if (st != FGFP8_OK) return st;
+  if (!scale) return fail(FGFP8_ERR_INVALID_ARG, "scale is NULL");
+  if (!aligned(scale, 4)) return fail(FGFP8_ERR_ALIGN, "scale must be 4-byte aligned");
+  int dev;
+  DeviceInfo info;
+  st = current_device(&dev, &info);
+  if (st != FGFP8_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t* word = reinterpret_cast<uint32_t*>(scale);
+  cudaError_t e = cudaMemsetAsync(word, 0, sizeof(uint32_t), s);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the amax word");
+  if (R > 0) {
+    fgfp8::FastDiv chunks(static_cast<uint32_t>(K / 8));
+    fgfp8::tensor_amax_kernel<<<grid_stride_blocks(R * (K / 8), info.sm_count), 256, 0, s>>>(
+        reinterpret_cast<const uint16_t*>(X), static_cast<uint32_t>(R), static_cast<uint32_t>(K),
+        static_cast<uint64_t>(ldx), chunks, word);
+    st = check_launch("tensor amax launch");
+    if (st != FGFP8_OK) return st;
+  }
+  fgfp8::tensor_scale_finish_kernel<<<1, 32, 0, s>>>(word);
+  return check_launch("tensor scale launch");
+}
+
+fgfp8_status fgfp8_quant_static(const void* X, int64_t R, int64_t K, int64_t ldx, const float* scale, uint8_t* Xq,
+                                void* stream) {
+  fgfp8_status st = check_rows_common(X, R, K, ldx, true, Xq);
+  if (st != FGFP8_OK) return st;
+  if (R == 0) return ok();
+  if (!scale) return fail(FGFP8_ERR_INVALID_ARG, "scale is NULL");
+  if (!aligned(scale, 4)) return fail(FGFP8_ERR_ALIGN, "scale must be 4-byte aligned");
+  int dev;
+  DeviceInfo info;
+  st = current_device(&dev, &info);
+  if (st != FGFP8_OK) return st;
+  fgfp8::FastDiv chunks(static_cast<uint32_t>(K / 8));
+  fgfp8::quant_static_kernel<<<grid_stride_blocks(R * (K / 8), info.sm_count), 256, 0,
+                               reinterpret_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint16_t*>(X), static_cast<uint32_t>(R), static_cast<uint32_t>(K),
+      static_cast<uint64_t>(ldx), chunks, scale, Xq);
+  return check_launch("quant_static launch");
+}
+
+fgfp8_status fgfp8_gemm_rowcol(const uint8_t* Xq, const float* sx, int x_per_tensor, const uint8_t* Wq,
+                               const float* sw, int w_per_tensor, void* Y, int64_t M, int64_t N, int64_t K,
+                               void* stream) {
+  if (x_per_tensor != 0 && x_per_tensor != 1) return fail(FGFP8_ERR_INVALID_ARG, "x_per_tensor must be 0 or 1");
+  if (w_per_tensor != 0 && w_per_tensor != 1) return fail(FGFP8_ERR_INVALID_ARG, "w_per_tensor must be 0 or 1");
+  if (M < 0 || N < 0 || K < 0) return fail(FGFP8_ERR_INVALID_ARG, "negative size");
+  if (K == 0 || K % 128 != 0) return fail(FGFP8_ERR_SHAPE, "K must be a positive multiple of 128");
+  if (N == 0 || N % 128 != 0) return fail(FGFP8_ERR_SHAPE, "N must be a positive multiple of 128");
+  if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+    return fail(FGFP8_ERR_SHAPE, "M, N and K must be < 2^31");
+  if (M == 0) return ok();
+  if (!Xq || !Wq || !sx || !sw || !Y) return fail(FGFP8_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned(Xq, 16) || !aligned(Wq, 16) || !aligned(Y, 16))
+    return fail(FGFP8_ERR_ALIGN, "Xq, Wq and Y must be 16-byte aligned");
+  if (!aligned(sx, 4)) return fail(FGFP8_ERR_ALIGN, "sx must be 4-byte aligned");
+  if (!aligned(sw, w_per_tensor ? 4 : 16))
+    return fail(FGFP8_ERR_ALIGN, "per-channel sw must be 16-byte aligned (4 bytes for one per-tensor scale)");
+  int dev;
+  DeviceInfo info;
+  fgfp8_status st = current_device(&dev, &info);
+  if (st != FGFP8_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (N % 256 == 0)
+    return launch_gemm_rowcol<256>(Xq, sx, x_per_tensor, Wq, sw, w_per_tensor, Y, M, N, K, s, dev, info.sm_count);
+  return launch_gemm_rowcol<128>(Xq, sx, x_per_tensor, Wq, sw, w_per_tensor, Y, M, N, K, s, dev, info.sm_count);
 }
 
 fgfp8_status fgfp8_check_device_status(void* stream) {

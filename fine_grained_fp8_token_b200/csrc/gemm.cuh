@@ -846,6 +846,221 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
+// Row/column-scaled GEMM ("FP8 W8A8", "Applying quantization": the
+// FP8_DYNAMIC scheme, per-output-channel weight scales and per-token
+// activation scales; or one static scale for a whole tensor):
+//   Y[m, n] = bf16( sx[m] * sw[n] * sum_k Xq[m, k] * Wq[n, k] )
+// with sx[0] for every m when x_per_tensor, sw[0] for every n when
+// w_per_tensor.  No scale changes along K, so the whole K reduction
+// accumulates in TMEM and the scales are applied once, in the epilogue:
+//   warp 0      TMA producer: one 128x128 Xq tile and one BNx128 Wq tile per
+//               K block into a kStages ring (128-byte swizzle);
+//   warp 1      TMEM owner and MMA issuer: four K=32 tcgen05.mma
+//               (kind::f8f6f4) per K block into the tile's accumulator; two
+//               accumulators, so one tile's epilogue overlaps the next tile's
+//               MMAs;
+//   warps 4..   epilogue: each thread one row and 128 columns; TMEM ->
+//               registers, times sx[m] * sw[n] (an fp32 product, then an fp32
+//               multiply), bf16 (round-to-nearest-even), global.
+// ---------------------------------------------------------------------------
+template <int BN>
+struct RowColCfg {
+  static constexpr int kBM = 128, kBN = BN, kBK = 128;
+  static constexpr int kEpiWarps = 4 * (BN / 128);
+  static constexpr int kThreads = 128 + 32 * kEpiWarps;
+  static constexpr int kNumAcc = 2;
+  static constexpr uint32_t kABytes = kBM * kBK;
+  static constexpr uint32_t kBBytes = kBN * kBK;
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = (BN == 128) ? 6 : 4;
+  static constexpr uint32_t kTmemCols = kNumAcc * BN;
+  static constexpr size_t kSmemBytes = 1024 + kStages * static_cast<size_t>(kStageBytes) + 256;
+};
+
+template <int BN>
+__global__ void __launch_bounds__(RowColCfg<BN>::kThreads, 1)
+    gemm_rowcol_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                       const float* __restrict__ sx, int x_per_tensor, const float* __restrict__ sw,
+                       int w_per_tensor, __nv_bfloat16* __restrict__ Y, int M, int N, int K, int num_tiles) {
+  using C = RowColCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + C::kStages * C::kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::kStages * C::kBBytes);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* mma_done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int KB = K / C::kBK;
+  const int num_m = (M + C::kBM - 1) / C::kBM;
+  // tile t -> (m0, n0), M-fastest
+  auto coords = [&](int t, int& m0, int& n0) {
+    m0 = (t % num_m) * C::kBM;
+    n0 = (t / num_m) * C::kBN;
+  };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], C::kEpiWarps);
+    }
+    mbar_init(mma_done, 1);
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  // programmatic launch: every access follows the preceding grid
+  griddep_wait();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ================= TMA producer
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        int m0, n0;
+        coords(t, m0, n0);
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % C::kStages;
+          if (it >= static_cast<uint32_t>(C::kStages) && !mbar_wait(&empty[s], ((it / C::kStages) & 1u) ^ 1u)) {
+            record_status(kDevTimeoutProducer);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+          tma_load_2d(sB + s * C::kBBytes, &tmB, &full[s], kb * C::kBK, n0);
+          tma_load_2d(sA + s * C::kABytes, &tmA, &full[s], kb * C::kBK, m0);
+        }
+      }
+      // every copy issued must land before the CTA may exit
+      for (uint32_t j = (it > static_cast<uint32_t>(C::kStages) ? it - C::kStages : 0); j < it; ++j)
+        if (!mbar_wait(&full[j % C::kStages], (j / C::kStages) & 1u)) record_status(kDevTimeoutProducer);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ================= MMA issuer
+      constexpr uint32_t idesc = idesc_e4m3_f32(128, C::kBN);
+      const uint64_t a_desc0 = smem_desc_k_sw128(smem_u32(sA)), b_desc0 = smem_desc_k_sw128(smem_u32(sB));
+      uint32_t it = 0, tile_no = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++tile_no) {
+        const int ab = tile_no & 1;                      // accumulator and its tfull / tempty barriers
+        if (tile_no >= 2 && !mbar_wait(&tempty[ab], ((tile_no - 2) >> 1) & 1u)) {
+          record_status(kDevTimeoutMma);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(ab * C::kBN);
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % C::kStages;
+          if (!mbar_wait(&full[s], (it / C::kStages) & 1u)) {
+            record_status(kDevTimeoutMma);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t adesc = a_desc0 + ((s * C::kABytes + kk * 32) >> 4);
+            const uint64_t bdesc = b_desc0 + ((s * C::kBBytes + kk * 32) >> 4);
+            mma_f8f6f4(d, adesc, bdesc, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&empty[s]);
+        }
+        if (ok) mma_commit(&tfull[ab]);
+      }
+      mma_commit(mma_done);
+      if (!mbar_wait(mma_done, 0)) record_status(kDevTimeoutMma);
+    }
+  } else if (warp >= 4) {
+    // ================= epilogue: TMEM -> scales -> bf16 -> global
+    const int ew = warp - 4;
+    const int quad = warp & 3;
+    const int col0 = (ew >> 2) * 128;
+    const int row = quad * 32 + lane;
+    uint32_t tile_no = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++tile_no) {
+      int m0, n0;
+      coords(t, m0, n0);
+      const int ab = tile_no & 1;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[ab], (tile_no >> 1) & 1u))) {
+        if (lane == 0) record_status(kDevTimeoutEpilogue);
+        break;
+      }
+      tc_fence_after();
+      const int m = m0 + row;
+      const uint32_t taddr =
+          tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(ab * C::kBN + col0);
+      // the whole 128-column slice into registers, then the accumulator is
+      // handed back before the scale multiplies and the stores
+      uint32_t p[128];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) tmem_ld_32x32b_x32(taddr + h * 32, *reinterpret_cast<uint32_t(*)[32]>(&p[h * 32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[ab]);
+      if (m < M) {
+        const float a = __ldg(sx + (x_per_tensor ? 0 : m));
+        const float w0 = w_per_tensor ? __ldg(sw) : 0.0f;
+        __nv_bfloat16* yrow = Y + static_cast<uint64_t>(m) * N + n0 + col0;
+        const float4* swv = reinterpret_cast<const float4*>(sw + n0 + col0);
+#pragma unroll
+        for (int j = 0; j < 128; j += 8) {
+          float c[8];
+          if (w_per_tensor) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) c[i] = __fmul_rn(a, w0);
+          } else {
+            const float4 u = __ldg(swv + j / 4), v = __ldg(swv + j / 4 + 1);
+            c[0] = __fmul_rn(a, u.x); c[1] = __fmul_rn(a, u.y); c[2] = __fmul_rn(a, u.z); c[3] = __fmul_rn(a, u.w);
+            c[4] = __fmul_rn(a, v.x); c[5] = __fmul_rn(a, v.y); c[6] = __fmul_rn(a, v.z); c[7] = __fmul_rn(a, v.w);
+          }
+          uint4 o;
+          __nv_bfloat162 h0 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(p[j + 0]), c[0]),
+                                                    __fmul_rn(__uint_as_float(p[j + 1]), c[1]));
+          __nv_bfloat162 h1 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(p[j + 2]), c[2]),
+                                                    __fmul_rn(__uint_as_float(p[j + 3]), c[3]));
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(p[j + 4]), c[4]),
+                                                    __fmul_rn(__uint_as_float(p[j + 5]), c[5]));
+          __nv_bfloat162 h3 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(p[j + 6]), c[6]),
+                                                    __fmul_rn(__uint_as_float(p[j + 7]), c[7]));
+          o.x = *reinterpret_cast<uint32_t*>(&h0);
+          o.y = *reinterpret_cast<uint32_t*>(&h1);
+          o.z = *reinterpret_cast<uint32_t*>(&h2);
+          o.w = *reinterpret_cast<uint32_t*>(&h3);
+          *reinterpret_cast<uint4*>(yrow + j) = o;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+// ---------------------------------------------------------------------------
 // Few-token variant (M <= 64, decode): operands swapped so the weight supplies
 // the MMA's 128 rows and the tokens its N dimension (BNT = M rounded up to
 // 16/32/64).  One CTA streams one 128-row weight slab through a deep TMA ring

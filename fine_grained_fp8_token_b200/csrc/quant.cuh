@@ -234,4 +234,106 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(const uint16_t* __res
   }
 }
 
+// ---------------------------------------------------------------------------
+// Row and tensor scale granularity ("FP8 W8A8", "Applying quantization": the
+// FP8_DYNAMIC scheme, per-output-channel weights and per-token activations;
+// static per-tensor AbsMax scales).  The scale and code rules are those of
+// the 1x128 groups above, with the group widened to a whole row of K or to
+// the whole tensor; scales are fp32.
+// ---------------------------------------------------------------------------
+
+// One CTA of kRowThreads per row r of X [R, K]: pass 1 takes the row's amax
+// (the first kRowRegChunks 16-byte chunks of each thread stay in registers),
+// the CTA reduces it, pass 2 writes the codes (chunks beyond the register
+// cache are read again, from L2).  Thread 0 stores the row's scale.
+constexpr int kRowThreads = 256;
+constexpr int kRowRegChunks = 8;     // rows up to 256 * 8 * 8 = 16384 elements in one read
+
+__global__ void __launch_bounds__(kRowThreads) quant_rows_kernel(const uint16_t* __restrict__ X, uint32_t K,
+                                                                 uint64_t ldx, uint8_t* __restrict__ Xq,
+                                                                 float* __restrict__ scales) {
+  __shared__ uint32_t s_max[kRowThreads / 32];
+  griddep_launch_dependents();
+  const uint32_t r = blockIdx.x;
+  const uint16_t* xr = X + static_cast<uint64_t>(r) * ldx;
+  uint8_t* qr = Xq + static_cast<uint64_t>(r) * K;
+  const uint32_t chunks = K / 8;                       // 16-byte chunks in the row
+  uint4 v[kRowRegChunks];
+  uint32_t a = 0;
+#pragma unroll
+  for (int i = 0; i < kRowRegChunks; ++i) {
+    const uint32_t c = threadIdx.x + i * kRowThreads;
+    if (c < chunks) {
+      v[i] = ld_stream_v4(xr + c * 8u);
+      a = max(a, absmax_bits8(v[i]));
+    }
+  }
+  for (uint32_t c = threadIdx.x + kRowRegChunks * kRowThreads; c < chunks; c += kRowThreads)
+    a = max(a, absmax_bits8(ld_stream_v4(xr + c * 8u)));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = max(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+  if ((threadIdx.x & 31u) == 0) s_max[threadIdx.x >> 5] = a;
+  __syncthreads();
+  a = s_max[0];
+#pragma unroll
+  for (int i = 1; i < kRowThreads / 32; ++i) a = max(a, s_max[i]);
+  const GroupScale gs = make_scale<0>(a);
+#pragma unroll
+  for (int i = 0; i < kRowRegChunks; ++i) {
+    const uint32_t c = threadIdx.x + i * kRowThreads;
+    if (c < chunks) *reinterpret_cast<uint2*>(qr + c * 8u) = quant8<0>(v[i], gs);
+  }
+  for (uint32_t c = threadIdx.x + kRowRegChunks * kRowThreads; c < chunks; c += kRowThreads)
+    *reinterpret_cast<uint2*>(qr + c * 8u) = quant8<0>(ld_stream_v4(xr + c * 8u), gs);
+  if (threadIdx.x == 0) scales[r] = gs.s;
+}
+
+// amax over a whole tensor: each thread folds 16-byte chunks of its
+// grid-stride share, the warp reduces, lane 0 raises *amax_bits (bf16
+// magnitude bits; NaN patterns order above infinity) with atomicMax.
+// *amax_bits must be zero beforehand.
+__global__ void __launch_bounds__(256) tensor_amax_kernel(const uint16_t* __restrict__ X, uint32_t R, uint32_t K,
+                                                          uint64_t ldx, FastDiv chunk_div,
+                                                          uint32_t* __restrict__ amax_bits) {
+  const uint32_t total = R * chunk_div.d;              // 16-byte chunks
+  uint32_t a = 0;
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+    const uint32_t row = chunk_div.div(i);
+    const uint32_t c = i - row * chunk_div.d;
+    a = max(a, absmax_bits8(ld_stream_v4(X + static_cast<uint64_t>(row) * ldx + c * 8u)));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = max(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+  if ((threadIdx.x & 31u) == 0 && a != 0u) atomicMax(amax_bits, a);
+}
+
+// The tensor's scale from its amax bits, in place: the word holding the
+// bits becomes the fp32 scale max(amax, 1e-4) / 448.
+__global__ void tensor_scale_finish_kernel(uint32_t* __restrict__ word) {
+  if (threadIdx.x == 0 && blockIdx.x == 0) {
+    const GroupScale gs = make_scale<0>(*word);
+    *reinterpret_cast<float*>(word) = gs.s;
+  }
+}
+
+// Static quantization with a given fp32 scale *scale (device):
+// code = E4M3(x / scale) over X [R, K], 16 bytes of input per thread step.
+__global__ void __launch_bounds__(256) quant_static_kernel(const uint16_t* __restrict__ X, uint32_t R, uint32_t K,
+                                                           uint64_t ldx, FastDiv chunk_div,
+                                                           const float* __restrict__ scale,
+                                                           uint8_t* __restrict__ Xq) {
+  griddep_launch_dependents();
+  GroupScale gs;
+  gs.s = __ldg(scale);
+  gs.r = __frcp_rn(gs.s);
+  gs.e8 = 0;
+  const uint32_t total = R * chunk_div.d;
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+    const uint32_t row = chunk_div.div(i);
+    const uint32_t c = i - row * chunk_div.d;
+    const uint4 v = ld_stream_v4(X + static_cast<uint64_t>(row) * ldx + c * 8u);
+    *reinterpret_cast<uint2*>(Xq + static_cast<uint64_t>(row) * K + c * 8u) = quant8<0>(v, gs);
+  }
+}
+
 }  // namespace fgfp8

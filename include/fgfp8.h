@@ -162,6 +162,62 @@ fgfp8_status fgfp8_grouped_linear(const void* X, int64_t ldx, uint8_t* Xq, void*
                                   const uint8_t* Wq, const void* Ws, void* Y, const int32_t* group_offs,
                                   int32_t E, int64_t M_total, int64_t N, int64_t K, int fmt, void* stream);
 
+/*
+ * Scale granularity per row or per tensor ("FP8 W8A8", "Applying
+ * quantization": the FP8_DYNAMIC scheme quantizes weights statically per
+ * output channel and activations dynamically per token; static activation
+ * scales, "Fine-grained FP8", "DeepGEMM fast path"; AbsMax per-tensor
+ * calibration on the OwLite FP8 page).  Scales are fp32 and follow the same
+ * rules as the 1x128 groups: scale = max(amax, 1e-4) / 448, code =
+ * E4M3(x / scale) rounded to nearest even and saturated.
+ */
+
+/*
+ * One scale per row of X bf16 [R, K] (row stride ldx elements, ldx % 8 == 0,
+ * 16-byte aligned): per-token activations (rows = tokens) or per-output-
+ * channel weights (rows = output channels of W [N, K]).
+ *   Xq      E4M3 codes [R, K], row stride K bytes, 16-byte aligned.
+ *   scales  float [R]: scales[r] = max(amax of row r, 1e-4) / 448.
+ * K % 128 == 0; R == 0 is a no-op.
+ */
+fgfp8_status fgfp8_quant_rows(const void* X, int64_t R, int64_t K, int64_t ldx, uint8_t* Xq, float* scales,
+                              void* stream);
+
+/*
+ * Per-tensor AbsMax scale of X bf16 [R, K]: *scale = max(amax over every
+ * element, 1e-4) / 448 (one float in device memory, written on `stream`; a
+ * NaN element gives a NaN scale).  The float is used as the reduction's
+ * working word until the final value is written.
+ */
+fgfp8_status fgfp8_tensor_scale(const void* X, int64_t R, int64_t K, int64_t ldx, float* scale, void* stream);
+
+/*
+ * Static quantization with a given scale: Xq = E4M3(X / *scale), where
+ * *scale is one float in device memory (a calibrated activation scale, or
+ * the output of fgfp8_tensor_scale).  Layouts as for fgfp8_quant_rows.
+ */
+fgfp8_status fgfp8_quant_static(const void* X, int64_t R, int64_t K, int64_t ldx, const float* scale, uint8_t* Xq,
+                                void* stream);
+
+/*
+ * Row/column-scaled FP8 GEMM:
+ *   Y[m, n] = bf16( sx[m] * sw[n] * sum_k Xq[m, k] * Wq[n, k] )
+ *   Xq  E4M3 [M, K] row-major, 16-byte aligned.
+ *   sx  float [M] per-token scales (x_per_tensor = 0) or float [1]
+ *       (x_per_tensor = 1), 4-byte aligned.
+ *   Wq  E4M3 [N, K] row-major, 16-byte aligned.
+ *   sw  float [N] per-channel scales (w_per_tensor = 0, 16-byte aligned) or
+ *       float [1] (w_per_tensor = 1).
+ *   Y   bf16 [M, N] row-major, 16-byte aligned.
+ * K % 128 == 0, N % 128 == 0, M >= 0 arbitrary.  The K sum accumulates in
+ * fp32; the result is within |Y - Y_exact| <= 2^-7 |Y_exact| + 1e-4 sum_k
+ * |x_hat w_hat|.  Launched with programmatic stream serialization like
+ * fgfp8_gemm.
+ */
+fgfp8_status fgfp8_gemm_rowcol(const uint8_t* Xq, const float* sx, int x_per_tensor, const uint8_t* Wq,
+                               const float* sw, int w_per_tensor, void* Y, int64_t M, int64_t N, int64_t K,
+                               void* stream);
+
 /* Size of the static scratch of fgfp8_linear_noalloc: 32 MiB per device. */
 #define FGFP8_NOALLOC_SCRATCH_BYTES (32u << 20)
 

@@ -122,6 +122,36 @@ def test_linear_validates_both_halves_first():
     assert g(A, 256, A, A, 256, A, A, A, A, 4, 0, 256, 256, 1, None) == OK          # empty
 
 
+def test_row_and_tensor_scale_validation():
+    q, t, st = fg.fgfp8_quant_rows, fg.fgfp8_tensor_scale, fg.fgfp8_quant_static
+    # X, R, K, ldx, Xq, scales, stream
+    assert q(A, 4, 100, 100, A, A, None) == SHAPE                    # K % 128
+    assert q(A, 4, 256, 128, A, A, None) == SHAPE                    # ldx < K
+    assert q(A, 4, 256, 260, A, A, None) == ALIGN                    # ldx % 8
+    assert q(A, 4, 256, 256, A + 8, A, None) == ALIGN                # Xq alignment
+    assert q(A, 4, 256, 256, A, 0, None) == INVALID                  # NULL scales
+    assert q(A, 4, 256, 256, A, A + 2, None) == ALIGN                # scales alignment
+    assert q(A, 0, 256, 256, A, A, None) == OK                       # empty
+    assert t(A, 4, 256, 256, 0, None) == INVALID                     # NULL scale
+    assert t(A + 4, 4, 256, 256, A, None) == ALIGN                   # X alignment
+    assert st(A, 4, 256, 256, 0, A, None) == INVALID                 # NULL scale
+    assert st(A, 4, 256, 256, A, 0, None) == INVALID                 # NULL Xq
+    assert st(A, 0, 256, 256, A, A, None) == OK                      # empty
+
+
+def test_gemm_rowcol_validation():
+    g = fg.fgfp8_gemm_rowcol
+    # Xq, sx, x_per_tensor, Wq, sw, w_per_tensor, Y, M, N, K, stream
+    assert g(A, A, 0, A, A, 0, A, 4, 256, 100, None) == SHAPE        # K
+    assert g(A, A, 0, A, A, 0, A, 4, 200, 256, None) == SHAPE        # N
+    assert g(A, A, 2, A, A, 0, A, 4, 256, 256, None) == INVALID      # flag
+    assert g(A, A, 0, A, A + 4, 0, A, 4, 256, 256, None) == ALIGN    # per-channel sw must be 16-byte aligned
+    assert g(A, A + 2, 0, A, A, 0, A, 4, 256, 256, None) == ALIGN    # sx alignment
+    assert g(A, A, 0, A, 0, 1, A, 4, 256, 256, None) == INVALID      # NULL sw
+    assert g(A, A, 0, A, A, 0, A + 8, 4, 256, 256, None) == ALIGN    # Y
+    assert g(A, A, 0, A, A, 0, A, 0, 256, 256, None) == OK           # empty
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the behaviour without a GPU")
 def test_valid_call_without_gpu_fails_loudly():
     """No CPU fallback: a well-formed request on a machine without an
@@ -130,5 +160,7 @@ def test_valid_call_without_gpu_fails_loudly():
     assert "cuda" in fg.fgfp8_last_error_string().lower()
     assert fg.fgfp8_gemm(A, A, 4, A, A, A, 4, 256, 256, 0, None) == CUDA
     assert fg.fgfp8_linear(A, 256, A, A, 4, A, A, A, 4, 256, 256, 0, None) == CUDA
+    assert fg.fgfp8_quant_rows(A, 4, 256, 256, A, A, None) == CUDA
+    assert fg.fgfp8_gemm_rowcol(A, A, 0, A, A, 0, A, 4, 256, 256, None) == CUDA
     with pytest.raises(fg.FGFP8Error):
         fg._check(fg.fgfp8_quant_weight(A, 128, 256, 256, A, A, 0, None), "quant_weight")

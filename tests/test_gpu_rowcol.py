@@ -1,0 +1,132 @@
+"""GPU parity of the row / tensor scale granularity against the oracle: the
+FP8_DYNAMIC scheme ("FP8 W8A8", "Applying quantization": per-output-channel
+weights, per-token activations) and static per-tensor scales.
+
+Codes and scales bit-exact; GEMM outputs within |gpu - ref| <= 2^-7 |ref| +
+1e-4 sum_k |x_hat w_hat|.  The GPU path and the oracle quantize the same
+seeded bf16 inputs each on their own; the oracle's GEMM inputs are its own
+codes."""
+import numpy as np
+import pytest
+import torch
+
+import fine_grained_fp8_token_b200 as fg
+import oracle
+import workloads
+from parity import assert_codes_equal, assert_gemm_close, assert_scales_equal, bits16, require_gpu, to_np, y_to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dev():
+    d = require_gpu()
+    fg.load()
+    return d
+
+
+@pytest.mark.parametrize("R,K,kind", [(1, 128, "normal"), (7, 4096, "normal_outliers"), (33, 14336, "heavy_tail"),
+                                      (130, 384, "normal"), (3, 20480, "normal_outliers"), (300, 1024, "heavy_tail")])
+def test_quant_rows(dev, R, K, kind):
+    X = workloads.activations((R, K), kind, seed=R + K)
+    Xq, s = fg.quant_rows(X.to(dev))
+    fg.check_device_status()
+    Xq_r, s_r = oracle.quant_rows(bits16(X))
+    assert_codes_equal(to_np(Xq), Xq_r, f"row codes {R}x{K}")
+    assert_scales_equal(to_np(s), s_r, f"row scales {R}x{K}")
+
+
+def test_quant_rows_strided_input(dev):
+    R, K, ldx = 20, 1024, 1536
+    big = workloads.activations((R, ldx), "normal_outliers", seed=9).to(dev)
+    X = big[:, :K]
+    Xq, s = fg.quant_rows(X)
+    Xq_r, s_r = oracle.quant_rows(bits16(X))
+    assert_codes_equal(to_np(Xq), Xq_r, "strided row codes")
+    assert_scales_equal(to_np(s), s_r, "strided row scales")
+
+
+@pytest.mark.parametrize("R,K", [(1, 128), (64, 7168), (4096, 4096), (513, 640)])
+def test_tensor_scale_and_static_quant(dev, R, K):
+    X = workloads.activations((R, K), "normal_outliers", seed=3 * R + K)
+    Xd = X.to(dev)
+    s = fg.tensor_scale(Xd)
+    Xq = fg.quant_static(Xd, s)
+    fg.check_device_status()
+    s_r = oracle.tensor_scale(bits16(X))
+    assert to_np(s).view(np.uint32)[0] == np.float32(s_r).view(np.uint32), (float(s), float(s_r))
+    assert_codes_equal(to_np(Xq), oracle.quant_static(bits16(X), s_r), f"static codes {R}x{K}")
+    # a calibrated scale that is not the tensor's own: saturation and small codes
+    for given in (np.float32(0.0031), np.float32(1.7e-5)):
+        Xq2 = fg.quant_static(Xd, torch.tensor([given], device=dev))
+        assert_codes_equal(to_np(Xq2), oracle.quant_static(bits16(X), given), f"static codes, scale {given}")
+
+
+def test_tensor_scale_zero_and_nan(dev):
+    Z = torch.zeros((3, 256), dtype=torch.bfloat16, device=dev)
+    assert float(fg.tensor_scale(Z)) == float(np.float32(1e-4) / np.float32(448.0))
+    X = torch.ones((5, 256), dtype=torch.bfloat16, device=dev)
+    X[4, 17] = float("nan")
+    assert torch.isnan(fg.tensor_scale(X)).all()
+
+
+def make_operands(dev, M, N, K, x_tensor, w_tensor, seed):
+    X = workloads.activations((M, K), "normal_outliers", seed=seed)
+    W = workloads.weights((N, K), seed=seed + 1)
+    Xd, Wd = X.to(dev), W.to(dev)
+    if x_tensor:
+        sx = fg.tensor_scale(Xd)
+        Xq = fg.quant_static(Xd, sx)
+        sx_r = np.array([oracle.tensor_scale(bits16(X))], dtype=np.float32)
+        Xq_r = oracle.quant_static(bits16(X), sx_r[0])
+    else:
+        Xq, sx = fg.quant_rows(Xd)
+        Xq_r, sx_r = oracle.quant_rows(bits16(X))
+    if w_tensor:
+        sw = fg.tensor_scale(Wd)
+        Wq = fg.quant_static(Wd, sw)
+        sw_r = np.array([oracle.tensor_scale(bits16(W))], dtype=np.float32)
+        Wq_r = oracle.quant_static(bits16(W), sw_r[0])
+    else:
+        Wq, sw = fg.quant_rows(Wd)
+        Wq_r, sw_r = oracle.quant_rows(bits16(W))
+    return (Xq, sx, Wq, sw), (Xq_r, sx_r, Wq_r, sw_r)
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 512), (300, 640, 2048), (1, 1280, 7168), (513, 384, 1024),
+                                   (64, 2304, 4096), (1200, 4096, 256)])
+@pytest.mark.parametrize("x_tensor,w_tensor", [(0, 0), (1, 0), (0, 1), (1, 1)])
+def test_gemm_rowcol(dev, M, N, K, x_tensor, w_tensor):
+    (Xq, sx, Wq, sw), (Xq_r, sx_r, Wq_r, sw_r) = make_operands(dev, M, N, K, x_tensor, w_tensor, seed=M + 7 * N + K)
+    Y = fg.gemm_rowcol(Xq, sx, Wq, sw)
+    fg.check_device_status()
+    Y_ref, S = oracle.gemm_rowcol(Xq_r, sx_r, Wq_r, sw_r)
+    assert_gemm_close(y_to_f64(Y), Y_ref, S, f"rowcol {M}x{N}x{K} x_tensor={x_tensor} w_tensor={w_tensor}")
+
+
+def test_gemm_rowcol_full_size_sampled_rows(dev):
+    """The Llama-3-8B attention projection in the FP8_DYNAMIC scheme, every
+    M tile's first and last row plus random rows against the oracle."""
+    cfg = workloads.LLAMA_ATTN
+    X = workloads.activations((cfg.M, cfg.K), cfg.x_kind, cfg.seed, device=dev)
+    W = workloads.weights((cfg.N, cfg.K), cfg.seed + 1, device=dev)
+    Xq, sx = fg.quant_rows(X)
+    Wq, sw = fg.quant_rows(W)
+    Y = fg.gemm_rowcol(Xq, sx, Wq, sw)
+    fg.check_device_status()
+    rng = np.random.default_rng(0)
+    tiles = np.arange(0, cfg.M, 128)
+    rows = np.unique(np.concatenate([tiles, tiles + 127, rng.integers(0, cfg.M, 32)]))
+    Xq_r, sx_r = oracle.quant_rows(bits16(X[torch.as_tensor(rows, device=dev)]))
+    Wq_r, sw_r = oracle.quant_rows(bits16(W))
+    Y_ref, S = oracle.gemm_rowcol(Xq_r, sx_r, Wq_r, sw_r)
+    assert_gemm_close(y_to_f64(Y[torch.as_tensor(rows, device=dev)]), Y_ref, S, "FP8_DYNAMIC 4096^3")
+
+
+def test_gemm_rowcol_empty_and_repeatable(dev):
+    (Xq, sx, Wq, sw), _ = make_operands(dev, 200, 512, 1024, 0, 0, seed=1)
+    Y1 = fg.gemm_rowcol(Xq, sx, Wq, sw)
+    Y2 = fg.gemm_rowcol(Xq, sx, Wq, sw)
+    assert torch.equal(Y1, Y2)
+    Y0 = fg.gemm_rowcol(Xq[:0], sx[:0], Wq, sw)
+    assert Y0.shape == (0, 512)
