@@ -11,7 +11,10 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def test_fastdiv_and_exact_quotient(tmp_path):
     exe = tmp_path / "host_checks"
     nvcc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "bin", "nvcc")
-    subprocess.run([nvcc, "-O2", "-std=c++17", "-Xcompiler", "-fopenmp,-ffp-contract=off,-fno-fast-math",
+    # the included kernel headers hold sm_100a device code (programmatic
+    # launch, cache-hinted loads): compile their device side for that target
+    subprocess.run([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-O2", "-std=c++17",
+                    "-Xcompiler", "-fopenmp,-ffp-contract=off,-fno-fast-math",
                     "-I", os.path.join(ROOT, "fine_grained_fp8_token_b200", "csrc"),
                     "-o", str(exe), os.path.join(ROOT, "tests", "host", "host_checks.cu"), "-lgomp"],
                    check=True)

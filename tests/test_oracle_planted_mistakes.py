@@ -37,8 +37,14 @@ MUTANTS = {
     "gemm_weight_scale_transposed": (
         "double sw = scale_at(Ws, ws_off + (n / ORC_GROUP) * KB + kb, fmt);",
         "double sw = scale_at(Ws, ws_off + kb * NB + n / ORC_GROUP, fmt);"),
-    "gemm_abs_weight": ("double prod = table[xr[k]] * table[wr[k]];",
-                        "double prod = table[xr[k]] * fabs(table[wr[k]]);"),
+    "gemm_abs_weight": ("for (int64_t k = kb * ORC_GROUP; k < (kb + 1) * ORC_GROUP; ++k) {\n"
+                        "                    double prod = table[xr[k]] * table[wr[k]];",
+                        "for (int64_t k = kb * ORC_GROUP; k < (kb + 1) * ORC_GROUP; ++k) {\n"
+                        "                    double prod = table[xr[k]] * fabs(table[wr[k]]);"),
+    "rowcol_abs_weight": ("for (int64_t k = 0; k < K; ++k) {\n"
+                          "                double prod = table[xr[k]] * table[wr[k]];",
+                          "for (int64_t k = 0; k < K; ++k) {\n"
+                          "                double prod = table[xr[k]] * fabs(table[wr[k]]);"),
     "grouped_segment_boundary": ("if (offs[i] <= m && m < offs[i + 1]) { e = i; break; }",
                                  "if (offs[i] <= m && m <= offs[i + 1]) { e = i; break; }"),
     "row_amax_half_row": ("float s = orc_scale_f32(amax_clamped(xr, K, 0, 1));",
