@@ -69,7 +69,9 @@ WORKLOAD_ALIASES = {
     "llama_attn_static": f"{workloads.LLAMA_ATTN.name}_static_tensor",
     "llama_gate_up_dynamic": f"{workloads.LLAMA_GATE_UP.name}_fp8_dynamic",
     "llama_down_dynamic": f"{workloads.LLAMA_DOWN.name}_fp8_dynamic",
+    "llama_mlp_fused": "llama3_8b_mlp_8192x4096x14336_swiglu_fused",
 }
+MLP_NAME = "llama3_8b_mlp_8192x4096x14336_swiglu_fused"
 
 
 def measured_peaks():
@@ -315,6 +317,81 @@ class RowColLayer:
         return "gemm_rowcol_kernel"
 
 
+class MLPLayer:
+    """The Llama-3-8B MLP in prefill (X [8192, 4096], gate/up [2 x 14336,
+    4096], down [4096, 14336], fp32 block scales) as three kernels: the 1x128
+    activation quantizer, the gate/up GEMM fused with SiLU * up and the down
+    projection's quantizer (fgfp8_gemm_swiglu_quant: the bf16 [8192, 28672]
+    gate/up output is never written), and the down GEMM."""
+
+    M, K, I, N_DOWN = 8192, 4096, 14336, 4096
+    launches_per_step = 3
+
+    def __init__(self, dev):
+        import fine_grained_fp8_token_b200 as fg
+        self.fg, self.dev = fg, dev
+        c = workloads.LLAMA_GATE_UP
+        self.X = workloads.activations((self.M, self.K), c.x_kind, c.seed, device=dev)
+        Wg = workloads.weights((self.I, self.K), c.seed + 1, device=dev)
+        Wu = workloads.weights((self.I, self.K), c.seed + 2, device=dev)
+        self.W_gu = fg.interleave_gate_up(Wg, Wu)
+        del Wg, Wu
+        self.W_down = workloads.weights((self.N_DOWN, self.I), c.seed + 3, device=dev)
+        self.Wq_gu = torch.empty((2 * self.I, self.K), dtype=torch.uint8, device=dev)
+        self.Ws_gu = torch.empty((2 * self.I // 128, self.K // 128), dtype=torch.float32, device=dev)
+        self.Wq_d = torch.empty((self.N_DOWN, self.I), dtype=torch.uint8, device=dev)
+        self.Ws_d = torch.empty((self.N_DOWN // 128, self.I // 128), dtype=torch.float32, device=dev)
+        self.ld_s = fg.scale_rows(self.M, 0)
+        self.Xq = torch.empty((self.M, self.K), dtype=torch.uint8, device=dev)
+        self.Xs = torch.empty((self.K // 128, self.ld_s), dtype=torch.float32, device=dev)
+        self.Hq = torch.empty((self.M, self.I), dtype=torch.uint8, device=dev)
+        self.Hs = torch.empty((self.I // 128, self.ld_s), dtype=torch.float32, device=dev)
+        self.Y = torch.empty((self.M, self.N_DOWN), dtype=torch.bfloat16, device=dev)
+        self.quant_weight()
+        fg.quant_weight(self.W_down, 0, Wq=self.Wq_d, Ws=self.Ws_d)
+        self.W = self.W_gu
+
+    def quant_weight(self):
+        self.fg.quant_weight(self.W_gu, 0, Wq=self.Wq_gu, Ws=self.Ws_gu)
+
+    def quant_act(self, X=None):
+        self.fg.quant_act(self.X if X is None else X, 0, Xq=self.Xq, Xs=self.Xs, ld_s=self.ld_s)
+
+    def gemm(self):
+        self.fg.gemm_swiglu_quant(self.Xq, self.Xs, self.Wq_gu, self.Ws_gu, Hq=self.Hq, Hs=self.Hs, ld_h=self.ld_s)
+        self.fg.gemm(self.Hq, self.Hs, self.Wq_d, self.Ws_d, 0, Y=self.Y)
+
+    def linear(self, X=None):
+        self.quant_act(X)
+        self.gemm()
+
+    def flops(self):
+        return 2.0 * self.M * (2 * self.I) * self.K + 2.0 * self.M * self.N_DOWN * self.I
+
+    def act_bytes(self):
+        return 3.0 * self.M * self.K + 4.0 * self.M * self.K / 128
+
+    def gemm_bytes(self):
+        # operands read once, h written once and read once (codes and scales), Y written
+        h = self.M * self.I * (1 + 4.0 / 128)
+        return (self.M * self.K + 2 * self.I * self.K + self.N_DOWN * self.I + 4.0 * (self.M * self.K + 2 * self.I
+                * self.K + self.N_DOWN * self.I) / 128 / 128 + 2 * h + 2.0 * self.M * self.N_DOWN)
+
+    def weight_bytes(self):
+        return 3.0 * 2 * self.I * self.K + 4.0 * 2 * self.I * self.K / 16384
+
+    def describe(self):
+        return {"workload": MLP_NAME, "M": self.M, "K": self.K, "I": self.I, "N_down": self.N_DOWN,
+                "scales": "fp32 (1x128 activations, 128x128 weights)", "x": "normal_outliers",
+                "chain": "quant_act -> gate/up GEMM + SiLU*up + quant (fused) -> down GEMM"}
+
+    def host_io(self):
+        return self.X, self.Y
+
+    def gemm_kernel_name(self):
+        return "gemm_blockscaled_kernel (fused SwiGLU) + gemm_blockscaled_kernel"
+
+
 class MoELayer:
     """Grouped expert layer: routed token rows and pre-quantized experts."""
 
@@ -383,6 +460,8 @@ class MoELayer:
 
 def make_layer(name, dev):
     name = WORKLOAD_ALIASES.get(name, name)
+    if name == MLP_NAME:
+        return MLPLayer(dev)
     if name in ROWCOL:
         cfg, scheme = ROWCOL[name]
         return RowColLayer(cfg, scheme, dev)
@@ -421,7 +500,7 @@ def run_gpu(args, rank, world, dev):
     stream = torch.cuda.current_stream(dev)
     flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
-    launches_per_step = 2
+    launches_per_step = getattr(layer, "launches_per_step", 2)
 
     for _ in range(args.warmup):
         flush_l2(flush_w, flush_r)
@@ -524,6 +603,23 @@ class OracleSample:
         self.oracle = oracle
         name = WORKLOAD_ALIASES.get(name, name)
         self.scheme = None
+        if name == MLP_NAME:
+            c = workloads.LLAMA_GATE_UP
+            X = workloads.activations((MLPLayer.M, MLPLayer.K), c.x_kind, c.seed)[:rows]
+            Wg = workloads.weights((MLPLayer.I, MLPLayer.K), c.seed + 1)
+            Wu = workloads.weights((MLPLayer.I, MLPLayer.K), c.seed + 2)
+            Wd = workloads.weights((MLPLayer.N_DOWN, MLPLayer.I), c.seed + 3)
+            b = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+            self.scheme, self.fmt = "mlp", 0
+            self.X = b(X)
+            self.Wq_g, self.Ws_g = oracle.quant_weight(b(Wg), 0)
+            self.Wq_u, self.Ws_u = oracle.quant_weight(b(Wu), 0)
+            self.Wq_d, self.Ws_d = oracle.quant_weight(b(Wd), 0)
+            self.rows = self.X.shape[0]
+            self.N, self.K = MLPLayer.N_DOWN, MLPLayer.K
+            self.desc = (f"first {self.rows} of {MLPLayer.M} tokens through gate/up, SiLU * up, the 1x128 "
+                         f"quantizer and down")
+            return
         if name in ROWCOL:
             cfg, self.scheme = ROWCOL[name]
             X, W = workloads.linear_inputs(cfg)
@@ -556,6 +652,14 @@ class OracleSample:
         self.rows = self.X.shape[0]
 
     def step(self):
+        if self.scheme == "mlp":
+            Xq, Xs = self.oracle.quant_act(self.X, 0)
+            g, _ = self.oracle.gemm(Xq, Xs, self.Wq_g, self.Ws_g, 0)
+            u, _ = self.oracle.gemm(Xq, Xs, self.Wq_u, self.Ws_u, 0)
+            h = self.oracle.bf16_rne(self.oracle.silu_mul(g, u))
+            Hq, Hs = self.oracle.quant_act(h, 0)
+            self.oracle.gemm(Hq, Hs, self.Wq_d, self.Ws_d, 0)
+            return
         if self.scheme == "fp8_dynamic":
             Xq, sx = self.oracle.quant_rows(self.X)
             self.oracle.gemm_rowcol(Xq, sx, self.Wq, self.sw)
@@ -568,6 +672,8 @@ class OracleSample:
         self.oracle.gemm(Xq, Xs, self.Wq, self.Ws, self.fmt)
 
     def flops(self):
+        if self.scheme == "mlp":
+            return 2.0 * self.rows * (2 * MLPLayer.I * MLPLayer.K + MLPLayer.N_DOWN * MLPLayer.I)
         return 2.0 * self.rows * self.N * self.K
 
 
@@ -699,7 +805,8 @@ def main():
                                      "bytes": layer.weight_bytes()},
             "apart_sum_us": 1e3 * (r["quant_ms"] + r["gemm_ms"]),
         },
-        "step_call": ("fgfp8_grouped_linear" if isinstance(layer, MoELayer) else
+        "step_call": ("fgfp8_quant_act + fgfp8_gemm_swiglu_quant + fgfp8_gemm" if isinstance(layer, MLPLayer) else
+                      "fgfp8_grouped_linear" if isinstance(layer, MoELayer) else
                       ("fgfp8_quant_rows + fgfp8_gemm_rowcol" if getattr(layer, "scheme", None) == "fp8_dynamic"
                        else "fgfp8_quant_static + fgfp8_gemm_rowcol") if isinstance(layer, RowColLayer)
                       else "fgfp8_linear"),

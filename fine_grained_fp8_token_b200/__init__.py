@@ -41,6 +41,7 @@ SIGNATURES = {
     "fgfp8_tensor_scale": (_INT, [_P, _I64, _I64, _I64, _P, _P]),
     "fgfp8_quant_static": (_INT, [_P, _I64, _I64, _I64, _P, _P, _P]),
     "fgfp8_gemm_rowcol": (_INT, [_P, _P, _INT, _P, _P, _INT, _P, _I64, _I64, _I64, _P]),
+    "fgfp8_gemm_swiglu_quant": (_INT, [_P, _P, _I64, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]),
     "fgfp8_check_device_status": (_INT, [_P]),
 }
 
@@ -104,6 +105,7 @@ fgfp8_quant_rows = _raw("fgfp8_quant_rows")
 fgfp8_tensor_scale = _raw("fgfp8_tensor_scale")
 fgfp8_quant_static = _raw("fgfp8_quant_static")
 fgfp8_gemm_rowcol = _raw("fgfp8_gemm_rowcol")
+fgfp8_gemm_swiglu_quant = _raw("fgfp8_gemm_swiglu_quant")
 fgfp8_check_device_status = _raw("fgfp8_check_device_status")
 
 
@@ -277,6 +279,38 @@ def gemm_rowcol(Xq, sx, Wq, sw, Y=None, stream=None):
     _check(fgfp8_gemm_rowcol(Xq.data_ptr(), sx.data_ptr(), x_t, Wq.data_ptr(), sw.data_ptr(), w_t, Y.data_ptr(),
                              M, N, K, _stream(stream)), "fgfp8_gemm_rowcol")
     return Y
+
+
+# ---------------------------------------------------------------- fused SwiGLU MLP
+def interleave_gate_up(gate, up, block: int = 128):
+    """Stack gate and up [R, ...] into the [2R, ...] layout that
+    fgfp8_gemm_swiglu_quant takes: blocks of `block` rows alternating gate,
+    up.  Weights (bf16, or their E4M3 codes) use block=128; their
+    [I/128, K/128] block scales use block=1.  Pure data layout (a torch stack
+    and reshape)."""
+    import torch
+    R = gate.shape[0]
+    g = gate.reshape(R // block, block, *gate.shape[1:])
+    u = up.reshape(R // block, block, *up.shape[1:])
+    return torch.stack([g, u], dim=1).reshape(2 * R, *gate.shape[1:]).contiguous()
+
+
+def gemm_swiglu_quant(Xq, Xs, Wq_gu, Ws_gu, Hq=None, Hs=None, ld_h: int | None = None, stream=None):
+    """h = SiLU(gate) * up of the interleaved gate/up projection, quantized
+    per 1x128 group for the down projection (fp32 scales).  Returns (Hq uint8
+    [M, I], Hs float32 [I/128, ld_h])."""
+    import torch
+    M, K = Xq.shape
+    I = Wq_gu.shape[0] // 2
+    ld_h = scale_rows(M, SCALE_F32) if ld_h is None else ld_h
+    if Hq is None:
+        Hq = torch.empty((M, I), dtype=torch.uint8, device=Xq.device)
+    if Hs is None:
+        Hs = torch.empty((I // 128, ld_h), dtype=torch.float32, device=Xq.device)
+    _check(fgfp8_gemm_swiglu_quant(Xq.data_ptr(), Xs.data_ptr(), Xs.shape[1], Wq_gu.data_ptr(), Ws_gu.data_ptr(),
+                                   Hq.data_ptr(), Hs.data_ptr(), ld_h, M, I, K, _stream(stream)),
+           "fgfp8_gemm_swiglu_quant")
+    return Hq, Hs
 
 
 def check_device_status(stream=None) -> None:

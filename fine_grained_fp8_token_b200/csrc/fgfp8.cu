@@ -154,10 +154,13 @@ fgfp8_status check_act_scales(const void* Xs, int64_t ld_s, int64_t M, int fmt) 
 }
 
 // Launch one GEMM instantiation as a persistent grid (one CTA per SM at most).
-template <int BN, int CW, int FMT, bool kGrouped>
+// kFuse: the SwiGLU gate/up projection writing the down projection's
+// quantized input (Hq, Hs, ld_h) instead of Y.
+template <int BN, int CW, int FMT, bool kGrouped, bool kFuse = false>
 fgfp8_status launch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
                          void* Y, int64_t M, int64_t N, int64_t K, const int32_t* offs, int E, int64_t b_rows,
-                         cudaStream_t stream, int dev, int sm_count, int early) {
+                         cudaStream_t stream, int dev, int sm_count, int early, uint8_t* Hq = nullptr,
+                         float* Hs = nullptr, int64_t ld_h = 0) {
   using C = fgfp8::GemmCfg<BN, CW>;
   CUtensorMap mA, mB, mBh;
   fgfp8_status st = make_map_u8_sw128(&mA, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
@@ -170,7 +173,7 @@ fgfp8_status launch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const 
   st = make_map_u8_sw128(&mBh, Wq, static_cast<uint64_t>(b_rows), static_cast<uint64_t>(K), static_cast<uint64_t>(K),
                          BN / 2);
   if (st != FGFP8_OK) return st;
-  auto kernel = fgfp8::gemm_blockscaled_kernel<BN, CW, FMT, kGrouped>;
+  auto kernel = fgfp8::gemm_blockscaled_kernel<BN, CW, FMT, kGrouped, kFuse>;
   st = set_smem(reinterpret_cast<const void*>(kernel), C::kSmemBytes, dev);
   if (st != FGFP8_OK) return st;
   if (C::kRegSplit) {
@@ -192,7 +195,7 @@ fgfp8_status launch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const 
   // twice into one wave (2R <= grid), those R tiles run as 2R half tiles,
   // so that wave takes about half a tile's time instead of a whole one.
   int64_t num_full = tiles, items = tiles;
-  if (!kGrouped && BN == 256) {
+  if (!kGrouped && !kFuse && BN == 256) {
     const int64_t waves = tiles / grid, rest = tiles - waves * grid;
     if (waves >= 1 && rest > 0 && 2 * rest <= grid) {
       num_full = waves * grid;
@@ -202,7 +205,8 @@ fgfp8_status launch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const 
   return launch_dependent(kernel, static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, stream, "gemm launch", mA,
                           mB, mBh, Xs, static_cast<uint32_t>(ld_s), Ws, reinterpret_cast<__nv_bfloat16*>(Y),
                           static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), offs, E,
-                          static_cast<int>(items), static_cast<int>(num_full), early);
+                          static_cast<int>(items), static_cast<int>(num_full), early, Hq, Hs,
+                          static_cast<uint32_t>(ld_h));
 }
 
 // UE8M0 launch with hardware block scaling (persistent, 128 x BN tiles).
@@ -677,6 +681,25 @@ fgfp8_status fgfp8_gemm_rowcol(const uint8_t* Xq, const float* sx, int x_per_ten
   if (N % 256 == 0)
     return launch_gemm_rowcol<256>(Xq, sx, x_per_tensor, Wq, sw, w_per_tensor, Y, M, N, K, s, dev, info.sm_count);
   return launch_gemm_rowcol<128>(Xq, sx, x_per_tensor, Wq, sw, w_per_tensor, Y, M, N, K, s, dev, info.sm_count);
+}
+
+fgfp8_status fgfp8_gemm_swiglu_quant(const uint8_t* Xq, const float* Xs, int64_t ld_s, const uint8_t* Wq_gu,
+                                     const float* Ws_gu, uint8_t* Hq, float* Hs, int64_t ld_h, int64_t M, int64_t I,
+                                     int64_t K, void* stream) {
+  if (M < 0 || I < 0) return fail(FGFP8_ERR_INVALID_ARG, "negative size");
+  if (I == 0 || I % 128 != 0) return fail(FGFP8_ERR_SHAPE, "I must be a positive multiple of 128");
+  if (M == 0) return ok();
+  fgfp8_status st = check_gemm_common(Xq, Xs, ld_s, Wq_gu, Ws_gu, Hq, M, 2 * I, K, FGFP8_SCALE_F32);
+  if (st != FGFP8_OK) return st;
+  st = check_act_scales(Hs, ld_h, M, FGFP8_SCALE_F32);
+  if (st != FGFP8_OK) return st;
+  int dev;
+  DeviceInfo info;
+  st = current_device(&dev, &info);
+  if (st != FGFP8_OK) return st;
+  return launch_gemm<256, 128, 0, false, true>(Xq, Xs, ld_s, Wq_gu, Ws_gu, nullptr, M, 2 * I, K, nullptr, 1, 2 * I,
+                                               reinterpret_cast<cudaStream_t>(stream), dev, info.sm_count, 0, Hq, Hs,
+                                               ld_h);
 }
 
 fgfp8_status fgfp8_check_device_status(void* stream) {

@@ -34,6 +34,7 @@
 #include <type_traits>
 
 #include "ptx.cuh"
+#include "quant.cuh"
 
 namespace fgfp8 {
 
@@ -205,15 +206,27 @@ __device__ __forceinline__ void issue_mmas(uint32_t a_base, uint32_t b_base, int
 // and promoted by all promotion warps at CW/2 columns each.  The host uses
 // them when the last partial wave of full tiles fits twice into one wave, so
 // that wave takes about half as long.
-template <int BN, int CW, int FMT, bool kGrouped>
+//
+// kFuse (dense, fp32 scales, 128 x 256 tiles): the SwiGLU MLP's gate/up
+// projection fused with the down projection's activation quantizer.  The
+// weight holds gate and up rows interleaved in 128-row blocks (rows
+// [256 j, 256 j + 128) are gate rows 128 j.., the next 128 the up rows), so a
+// tile's columns [0, 128) are gate and [128, 256) up outputs for the
+// intermediate indices i0 = n0 / 2 .. i0 + 127.  Instead of Y the epilogue
+// writes the codes Hq [M, I] and MN-major scales Hs[(i0 / 128) * ld_h + m]
+// of h = SiLU(gate) * up: the up warp of each TMEM lane quadrant hands its
+// bf16 outputs to the gate warp through shared memory, and the gate warp's
+// thread then holds one token's whole 1 x 128 group of h.
+template <int BN, int CW, int FMT, bool kGrouped, bool kFuse = false>
 __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
     gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmBh, const void* __restrict__ Xs, uint32_t ld_s,
                             const void* __restrict__ Ws, __nv_bfloat16* __restrict__ Y, int M, int N, int K,
                             const int32_t* __restrict__ group_offs, int E, int num_tiles, int num_full,
-                            int early_b) {
+                            int early_b, uint8_t* __restrict__ Hq, float* __restrict__ Hs, uint32_t ld_h) {
   using C = GemmCfg<BN, CW>;
-  constexpr bool kHalfTiles = !kGrouped && BN == 256;
+  static_assert(!kFuse || (BN == 256 && CW == 128 && FMT == 0 && !kGrouped), "fused SwiGLU: dense fp32 256-wide");
+  constexpr bool kHalfTiles = !kGrouped && BN == 256 && !kFuse;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -224,7 +237,9 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
   uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + C::kNumBuf;
   uint64_t* mma_done = tempty + C::kNumBuf;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* xfull = mma_done + 1;                     // fused epilogue: halves exchanged, per quadrant
+  uint64_t* xempty = xfull + 4;                       // fused epilogue: half-row amax exchanged, per quadrant
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xempty + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -267,6 +282,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
       mbar_init(&tempty[b], C::kEpiWarps);
     }
     mbar_init(mma_done, 1);
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(&xfull[q], 64);                       // both warps of the quadrant's pair
+      mbar_init(&xempty[q], 64);
+    }
     fence_mbarrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -412,7 +431,99 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
     };
     int pref_t = -1;                           // tile whose first scale words are in the ring
     uint32_t bt = 0;
+    uint32_t xt = 0;                           // fused epilogue: tiles handed over so far
     bool ok = true;
+
+    // Fused SwiGLU epilogue (kFuse).  The gate warp (grp 0) and the up warp
+    // (grp 1) of quadrant `quad` hold the same 32 rows: gate columns and up
+    // columns of the same 128 intermediate indices.  They split the work by
+    // halves: the gate warp sends g for columns 64..127 and the up warp u for
+    // columns 0..63 through the quadrant's shared-memory region (bf16, 16-byte
+    // chunk c of lane l at position c ^ (l % 8)), each forms h = bf16(silu(g)
+    // * u) for its 64 columns with g, u the bf16-rounded outputs and silu(g) =
+    // g / (1 + exp(-g)) in fp32 (hardware exponential and divide, a few fp32
+    // ulps), the two half-row amax values meet through the region, and each
+    // warp quantizes its 64 values with the row's scale exactly as the
+    // activation quantizer does.  Both meetings are bounded mbarrier waits on
+    // which all 64 lanes of the pair arrive.
+    auto fused_swiglu_epilogue = [&](float2 (&acc2)[CW / 2], int m0, int n0) {
+      uint8_t* region = sStg + quad * 8192;       // [0, 4 KB): g half, [4, 8 KB): u half
+      const uint32_t par = xt & 1u;
+      // kGate: this is the gate warp (keeps columns 0..63, sends g of 64..127)
+      // or the up warp (keeps 64..127, sends u of 0..63).  Once read, the
+      // partner's half carries this warp's half-row amax (slot = lane).
+      auto run = [&](auto gate_tag) -> bool {
+        constexpr bool kGate = decltype(gate_tag)::value;
+        constexpr int kSend0 = kGate ? 32 : 0, kOwn0 = kGate ? 0 : 32;
+        uint8_t* out = region + (kGate ? 0 : 4096);
+        uint8_t* in = region + (kGate ? 4096 : 0);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint4 v;
+          uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            __nv_bfloat162 b = __floats2bfloat162_rn(acc2[kSend0 + 4 * c + q].x, acc2[kSend0 + 4 * c + q].y);
+            w[q] = *reinterpret_cast<uint32_t*>(&b);
+          }
+          *reinterpret_cast<uint4*>(out + lane * 128 + ((c ^ (lane & 7)) << 4)) = v;
+        }
+        mbar_arrive(&xfull[quad]);
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&xfull[quad], par))) return false;
+        uint32_t hw[32];                           // h of my 64 columns as bf16 pairs
+        uint32_t a2 = 0;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 v = *reinterpret_cast<const uint4*>(in + lane * 128 + ((c ^ (lane & 7)) << 4));
+          const uint32_t* w = reinterpret_cast<const uint32_t*>(&v);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float p0 = __uint_as_float(w[q] << 16), p1 = __uint_as_float(w[q] & 0xFFFF0000u);
+            const float o0 = __bfloat162float(__float2bfloat16_rn(acc2[kOwn0 + 4 * c + q].x));
+            const float o1 = __bfloat162float(__float2bfloat16_rn(acc2[kOwn0 + 4 * c + q].y));
+            const float g0 = kGate ? o0 : p0, g1 = kGate ? o1 : p1;
+            const float u0 = kGate ? p0 : o0, u1 = kGate ? p1 : o1;
+            const float s0 = __fdividef(g0, __fadd_rn(1.0f, __expf(-g0)));
+            const float s1 = __fdividef(g1, __fadd_rn(1.0f, __expf(-g1)));
+            __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(s0, u0), __fmul_rn(s1, u1));
+            hw[4 * c + q] = *reinterpret_cast<uint32_t*>(&h);
+            a2 = __vmaxu2(a2, hw[4 * c + q] & 0x7FFF7FFFu);
+          }
+        }
+        const uint32_t mine = max(a2 & 0xFFFFu, a2 >> 16);
+        __syncwarp();                              // every lane has read its row of `in`
+        reinterpret_cast<uint32_t*>(in)[lane] = mine;
+        mbar_arrive(&xempty[quad]);
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&xempty[quad], par))) return false;
+        // the partner's half-row amax sits in the half this warp sent; its next
+        // overwrite follows the next tile's first meeting
+        const uint32_t amax = max(mine, reinterpret_cast<const uint32_t*>(out)[lane]);
+        const int m = m0 + row;
+        if (m < M) {
+          const GroupScale gs = make_scale<0>(amax);
+          const int i0 = n0 / 2;
+          uint8_t* dst = Hq + static_cast<uint64_t>(m) * (N / 2) + i0 + (kGate ? 0 : 64);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint4 o;
+            o.x = quant4<0>(hw[8 * c + 0], hw[8 * c + 1], gs);
+            o.y = quant4<0>(hw[8 * c + 2], hw[8 * c + 3], gs);
+            o.z = quant4<0>(hw[8 * c + 4], hw[8 * c + 5], gs);
+            o.w = quant4<0>(hw[8 * c + 6], hw[8 * c + 7], gs);
+            *reinterpret_cast<uint4*>(dst + 16 * c) = o;
+          }
+          if (kGate) Hs[static_cast<uint64_t>(i0 / 128) * ld_h + m] = gs.s;
+        }
+        return true;
+      };
+      const bool done = (grp == 0) ? run(std::true_type{}) : run(std::false_type{});
+      if (!done) {
+        if (lane == 0) record_status(kDevTimeoutEpilogue);
+        ok = false;
+        return;
+      }
+      ++xt;
+    };
 
     // One work item with COLS columns per warp: per K block, the partial from
     // TMEM times sa * sw into the accumulators, then the bf16 epilogue.
@@ -478,6 +589,13 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
 #pragma unroll
           for (int d = 0; d < kScaleAhead; ++d) fetch(d, mn, liven, wsn, ra[d], rw[d]);
           pref_t = tn;
+        }
+      }
+
+      if constexpr (kFuse) {
+        if constexpr (COLS == CW) {
+          fused_swiglu_epilogue(acc2, m0, n0);
+          return;
         }
       }
 

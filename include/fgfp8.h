@@ -218,6 +218,34 @@ fgfp8_status fgfp8_gemm_rowcol(const uint8_t* Xq, const float* sx, int x_per_ten
                                const float* sw, int w_per_tensor, void* Y, int64_t M, int64_t N, int64_t K,
                                void* stream);
 
+/*
+ * The gate/up projection of a SwiGLU MLP (Llama-3-8B's MLP: gate/up
+ * [2I, K], then down [K_out, I]) fused with the down projection's dynamic
+ * activation quantizer ("Fine-grained FP8", introduction and "DeepGEMM fast
+ * path": 1x128 per-token groups, fp32 scales).  For every token m and
+ * intermediate index i:
+ *   g, u   = bf16_rne of the block-scaled GEMM outputs of the gate and up rows
+ *   h      = bf16_rne( silu(g) * u ),  silu(g) = g * (1 / (1 + exp(-g))) in fp32
+ *   Hq, Hs = fgfp8_quant_act of h (fp32 scales): codes [M, I] row-major and
+ *            MN-major scales Hs[(i / 128) * ld_h + m]
+ * so Hq / Hs feed fgfp8_gemm with the down-projection weight directly and
+ * the bf16 [M, 2I] output of the gate/up projection is never written.
+ *   Xq, Xs, ld_s  the block-quantized input [M, K] (fp32 scales).
+ *   Wq_gu         E4M3 [2I, K]: gate and up rows interleaved in 128-row
+ *                 blocks, rows [256 j, 256 j + 128) = gate rows [128 j, ..),
+ *                 rows [256 j + 128, 256 j + 256) = up rows [128 j, ..).
+ *   Ws_gu         float [2I/128, K/128], the 128x128 block scales in the same
+ *                 interleaved order.
+ *   Hq            E4M3 [M, I], 16-byte aligned; Hs, ld_h as for
+ *                 fgfp8_quant_act (fp32, ld_h >= M, ld_h % 4 == 0).
+ * I % 128 == 0, K % 128 == 0.  The codes equal fgfp8_quant_act of the h the
+ * unfused layer would compute from its bf16 gate/up output, up to that
+ * output's own GEMM rounding.
+ */
+fgfp8_status fgfp8_gemm_swiglu_quant(const uint8_t* Xq, const float* Xs, int64_t ld_s, const uint8_t* Wq_gu,
+                                     const float* Ws_gu, uint8_t* Hq, float* Hs, int64_t ld_h, int64_t M, int64_t I,
+                                     int64_t K, void* stream);
+
 /* Size of the static scratch of fgfp8_linear_noalloc: 32 MiB per device. */
 #define FGFP8_NOALLOC_SCRATCH_BYTES (32u << 20)
 

@@ -336,6 +336,17 @@ def gemm_rowcol(Xq, sx, Wq, sw, rows=None):
     return Y, S
 
 
+# ---------------------------------------------------------------- SwiGLU MLP
+def silu_mul(g, u) -> np.ndarray:
+    """h = SiLU(g) * u = g / (1 + exp(-g)) * u in fp64: the input of a SwiGLU
+    MLP's down projection (Llama-3-8B's MLP, whose down-projection input the
+    measured configurations model as a post-SiLU heavy-tailed activation)."""
+    g = np.asarray(g, dtype=np.float64)
+    u = np.asarray(u, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return g / (1.0 + np.exp(-g)) * u
+
+
 def gemm_within_tolerance(Y_test, Y_ref, S) -> np.ndarray:
     """Elementwise |Y_test - Y_ref| <= 2^-7 |Y_ref| + 1e-4 S (the stated GEMM
     tolerance).  Y_test may be fp32/fp64 or bf16 torch data."""

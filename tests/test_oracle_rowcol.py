@@ -160,3 +160,19 @@ def test_gemm_rowcol_all_ones():
     Wq[:, ::2] = 0xB8                               # -1.0 on even k: the sum cancels
     Y, S = orc.gemm_rowcol(Xq, np.ones(M, np.float32), Wq, np.full(N, 2.0, np.float32))
     assert (Y == 0).all() and (S == 2 * K).all()
+
+
+def test_silu_mul_against_torch_and_limits():
+    """SiLU(g) * u against torch's silu in float64 (a library routine), and the
+    closed forms SiLU(0) = 0, SiLU(g) -> g for large g, SiLU(g) -> 0 for very
+    negative g."""
+    import oracle as orc
+    rng = np.random.default_rng(2)
+    g = np.concatenate([rng.normal(0, 3, 5000), [0.0, 40.0, -40.0, 1e-8, -1e-8, 700.0, -745.0]])
+    u = rng.normal(0, 1, g.size)
+    h = orc.silu_mul(g, u)
+    ref = (torch.nn.functional.silu(torch.from_numpy(g)) * torch.from_numpy(u)).numpy()
+    assert np.allclose(h, ref, rtol=1e-15, atol=0)
+    assert orc.silu_mul(0.0, 5.0) == 0.0
+    assert abs(orc.silu_mul(40.0, 1.0) - 40.0) < 1e-15 * 40
+    assert abs(orc.silu_mul(-745.0, 1.0)) < 1e-300
