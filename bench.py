@@ -70,6 +70,7 @@ WORKLOAD_ALIASES = {
     "llama_gate_up_dynamic": f"{workloads.LLAMA_GATE_UP.name}_fp8_dynamic",
     "llama_down_dynamic": f"{workloads.LLAMA_DOWN.name}_fp8_dynamic",
     "llama_mlp_fused": "llama3_8b_mlp_8192x4096x14336_swiglu_fused",
+    "moe_decode_masked": workloads.MOE_DECODE.name,
 }
 MLP_NAME = "llama3_8b_mlp_8192x4096x14336_swiglu_fused"
 
@@ -392,6 +393,83 @@ class MLPLayer:
         return "gemm_blockscaled_kernel (fused SwiGLU) + gemm_blockscaled_kernel"
 
 
+class MaskedMoELayer:
+    """Decode step of the expert layer in the masked layout: 128 tokens
+    routed top-8 (Zipf-skewed) to 256 experts, every expert a fixed block of
+    cap = 128 rows of which the first counts[e] hold tokens; the step is the
+    1x128 quantizer over the whole [E * cap, K] buffer and fgfp8_masked_gemm.
+    Experts without tokens are skipped, so the GEMM streams the weights of
+    the active experts only."""
+
+    CAP = 128
+
+    def __init__(self, cfg: workloads.MoE, dev):
+        import fine_grained_fp8_token_b200 as fg
+        self.fg, self.cfg, self.dev = fg, cfg, dev
+        self.r = workloads.moe_routing(cfg)
+        self.X = workloads.moe_masked_rows(workloads.moe_tokens(cfg, device=dev), self.r, cfg.E, self.CAP)
+        sdt = torch.float32 if cfg.fmt == 0 else torch.uint8
+        self.Wq = torch.empty((cfg.E, cfg.N, cfg.K), dtype=torch.uint8, device=dev)
+        self.Ws = torch.empty((cfg.E, cfg.N // 128, cfg.K // 128), dtype=sdt, device=dev)
+        for e in range(cfg.E):
+            fg.quant_weight(workloads.moe_expert_weight(cfg, e, device=dev), cfg.fmt, Wq=self.Wq[e], Ws=self.Ws[e])
+        self.counts = torch.as_tensor(self.r.counts.astype(np.int32), device=dev)
+        M = cfg.E * self.CAP
+        self.ld_s = fg.scale_rows(M, cfg.fmt)
+        self.Xq = torch.empty((M, cfg.K), dtype=torch.uint8, device=dev)
+        self.Xs = torch.empty((cfg.K // 128, self.ld_s), dtype=sdt, device=dev)
+        self.Y = torch.empty((M, cfg.N), dtype=torch.bfloat16, device=dev)
+        self.W = workloads.moe_expert_weight(cfg, 0, device=dev)
+        self.active = int((self.r.counts > 0).sum())
+
+    def quant_weight(self):
+        self.fg.quant_weight(self.W, self.cfg.fmt, Wq=self.Wq[0], Ws=self.Ws[0])
+
+    def quant_act(self, X=None):
+        self.fg.quant_act(self.X if X is None else X, self.cfg.fmt, Xq=self.Xq, Xs=self.Xs, ld_s=self.ld_s)
+
+    def gemm(self):
+        self.fg.masked_gemm(self.Xq, self.Xs, self.Wq, self.Ws, self.counts, self.cfg.fmt, Y=self.Y)
+
+    def linear(self, X=None):
+        self.quant_act(X)
+        self.gemm()
+
+    def flops(self):
+        c = self.cfg
+        return 2.0 * float(self.r.counts.sum()) * c.N * c.K
+
+    def act_bytes(self):
+        c = self.cfg
+        M = c.E * self.CAP
+        return 3.0 * M * c.K + (4 if c.fmt == 0 else 1) * M * c.K / 128
+
+    def gemm_bytes(self):
+        # the active experts' weights and scales, the token rows' codes and scales, Y's token rows
+        c = self.cfg
+        rows = float(self.r.counts.sum())
+        sb = 4 if c.fmt == 0 else 1
+        return (self.active * c.N * c.K * (1 + sb / 16384.0) + rows * c.K * (1 + sb / 128.0)
+                + 2.0 * rows * c.N)
+
+    def weight_bytes(self):
+        c = self.cfg
+        return 3.0 * c.N * c.K + (4 if c.fmt == 0 else 1) * c.N * c.K / 16384
+
+    def describe(self):
+        c = self.cfg
+        return {"workload": c.name, "experts": c.E, "active_experts": self.active, "cap": self.CAP, "N": c.N,
+                "K": c.K, "tokens": c.tokens, "topk": c.topk, "zipf": c.zipf,
+                "rows_routed": int(self.r.counts.sum()), "max_rows_per_expert": int(self.r.counts.max()),
+                "scales": "fp32" if c.fmt == 0 else "ue8m0"}
+
+    def host_io(self):
+        return self.X, self.Y
+
+    def gemm_kernel_name(self):
+        return ("gemm_blockscaled_kernel" if self.cfg.fmt == 0 else "gemm_mx_kernel") + " (masked)"
+
+
 class MoELayer:
     """Grouped expert layer: routed token rows and pre-quantized experts."""
 
@@ -460,6 +538,8 @@ class MoELayer:
 
 def make_layer(name, dev):
     name = WORKLOAD_ALIASES.get(name, name)
+    if name == workloads.MOE_DECODE.name:
+        return MaskedMoELayer(workloads.MOE_DECODE, dev)
     if name == MLP_NAME:
         return MLPLayer(dev)
     if name in ROWCOL:
@@ -632,8 +712,9 @@ class OracleSample:
             self.desc = (f"first {self.rows} of {cfg.M} rows x the full [{cfg.N}, {cfg.K}] weight, "
                          f"{self.scheme} scales")
             return
-        if name in (workloads.MOE.name, workloads.MOE_SMALL.name):
-            cfg = workloads.MOE if name == workloads.MOE.name else workloads.MOE_SMALL
+        if name in (workloads.MOE.name, workloads.MOE_SMALL.name, workloads.MOE_DECODE.name):
+            cfg = {workloads.MOE.name: workloads.MOE, workloads.MOE_SMALL.name: workloads.MOE_SMALL,
+                   workloads.MOE_DECODE.name: workloads.MOE_DECODE}[name]
             r = workloads.moe_routing(cfg)
             e = int(np.argmax(r.counts))                    # the busiest expert's rows
             tok = r.row_token[r.group_offs[e]:r.group_offs[e] + r.counts[e]]
@@ -806,6 +887,7 @@ def main():
             "apart_sum_us": 1e3 * (r["quant_ms"] + r["gemm_ms"]),
         },
         "step_call": ("fgfp8_quant_act + fgfp8_gemm_swiglu_quant + fgfp8_gemm" if isinstance(layer, MLPLayer) else
+                      "fgfp8_quant_act + fgfp8_masked_gemm" if isinstance(layer, MaskedMoELayer) else
                       "fgfp8_grouped_linear" if isinstance(layer, MoELayer) else
                       ("fgfp8_quant_rows + fgfp8_gemm_rowcol" if getattr(layer, "scheme", None) == "fp8_dynamic"
                        else "fgfp8_quant_static + fgfp8_gemm_rowcol") if isinstance(layer, RowColLayer)

@@ -42,6 +42,7 @@ SIGNATURES = {
     "fgfp8_quant_static": (_INT, [_P, _I64, _I64, _I64, _P, _P, _P]),
     "fgfp8_gemm_rowcol": (_INT, [_P, _P, _INT, _P, _P, _INT, _P, _I64, _I64, _I64, _P]),
     "fgfp8_gemm_swiglu_quant": (_INT, [_P, _P, _I64, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]),
+    "fgfp8_masked_gemm": (_INT, [_P, _P, _I64, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _INT, _P]),
     "fgfp8_check_device_status": (_INT, [_P]),
 }
 
@@ -106,6 +107,7 @@ fgfp8_tensor_scale = _raw("fgfp8_tensor_scale")
 fgfp8_quant_static = _raw("fgfp8_quant_static")
 fgfp8_gemm_rowcol = _raw("fgfp8_gemm_rowcol")
 fgfp8_gemm_swiglu_quant = _raw("fgfp8_gemm_swiglu_quant")
+fgfp8_masked_gemm = _raw("fgfp8_masked_gemm")
 fgfp8_check_device_status = _raw("fgfp8_check_device_status")
 
 
@@ -278,6 +280,22 @@ def gemm_rowcol(Xq, sx, Wq, sw, Y=None, stream=None):
     w_t = int(sw.numel() == 1 and N != 1)
     _check(fgfp8_gemm_rowcol(Xq.data_ptr(), sx.data_ptr(), x_t, Wq.data_ptr(), sw.data_ptr(), w_t, Y.data_ptr(),
                              M, N, K, _stream(stream)), "fgfp8_gemm_rowcol")
+    return Y
+
+
+def masked_gemm(Xq, Xs, Wq, Ws, counts, fmt: int, Y=None, stream=None):
+    """Masked expert GEMM: Xq [E * cap, K] with expert e's tokens in rows
+    [e * cap, e * cap + counts[e]), Wq [E, N, K], Ws [E, N/128, K/128],
+    counts int32 [E] on the device.  Returns Y bf16 [E * cap, N] (padding
+    rows are not written)."""
+    import torch
+    M_total, K = Xq.shape
+    E, N, _ = Wq.shape
+    cap = M_total // E
+    if Y is None:
+        Y = torch.empty((M_total, N), dtype=torch.bfloat16, device=Xq.device)
+    _check(fgfp8_masked_gemm(Xq.data_ptr(), Xs.data_ptr(), Xs.shape[1], Wq.data_ptr(), Ws.data_ptr(), Y.data_ptr(),
+                             counts.data_ptr(), E, cap, N, K, fmt, _stream(stream)), "fgfp8_masked_gemm")
     return Y
 
 

@@ -159,7 +159,7 @@ fgfp8_status check_act_scales(const void* Xs, int64_t ld_s, int64_t M, int fmt) 
 template <int BN, int CW, int FMT, bool kGrouped, bool kFuse = false>
 fgfp8_status launch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
                          void* Y, int64_t M, int64_t N, int64_t K, const int32_t* offs, int E, int64_t b_rows,
-                         cudaStream_t stream, int dev, int sm_count, int early, uint8_t* Hq = nullptr,
+                         cudaStream_t stream, int dev, int sm_count, int early, int cap = 0, uint8_t* Hq = nullptr,
                          float* Hs = nullptr, int64_t ld_h = 0) {
   using C = fgfp8::GemmCfg<BN, CW>;
   CUtensorMap mA, mB, mBh;
@@ -204,7 +204,7 @@ fgfp8_status launch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const 
   }
   return launch_dependent(kernel, static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, stream, "gemm launch", mA,
                           mB, mBh, Xs, static_cast<uint32_t>(ld_s), Ws, reinterpret_cast<__nv_bfloat16*>(Y),
-                          static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), offs, E,
+                          static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), offs, E, cap,
                           static_cast<int>(items), static_cast<int>(num_full), early, Hq, Hs,
                           static_cast<uint32_t>(ld_h));
 }
@@ -213,7 +213,7 @@ fgfp8_status launch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const 
 template <int BN, bool kGrouped>
 fgfp8_status launch_gemm_mx(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
                             void* Y, int64_t M, int64_t N, int64_t K, const int32_t* offs, int E, int64_t b_rows,
-                            cudaStream_t stream, int dev, int sm_count, int early) {
+                            cudaStream_t stream, int dev, int sm_count, int early, int cap) {
   using C = fgfp8::MxCfg<BN>;
   CUtensorMap mA, mB;
   fgfp8_status st = make_map_u8_sw128(&mA, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
@@ -232,13 +232,13 @@ fgfp8_status launch_gemm_mx(const uint8_t* Xq, const void* Xs, int64_t ld_s, con
                           "block-scaled gemm launch", mA, mB, reinterpret_cast<const uint8_t*>(Xs),
                           static_cast<uint32_t>(ld_s), reinterpret_cast<const uint8_t*>(Ws),
                           reinterpret_cast<__nv_bfloat16*>(Y), static_cast<int>(M), static_cast<int>(N),
-                          static_cast<int>(K), offs, E, static_cast<int>(tiles), early);
+                          static_cast<int>(K), offs, E, cap, static_cast<int>(tiles), early);
 }
 
 template <bool kGrouped>
 fgfp8_status dispatch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws, void* Y,
                            int64_t M, int64_t N, int64_t K, int fmt, const int32_t* offs, int E, int64_t b_rows,
-                           cudaStream_t s, int dev, int sms, int early) {
+                           cudaStream_t s, int dev, int sms, int early, int cap = 0) {
   // 128x256 tiles: measured faster per FLOP than 128x128 on B200 even where
   // 128x128 tiles would fill the last wave better (4096^3: 95 us vs 119 us);
   // 128x128 only when N is not a multiple of 256.
@@ -249,12 +249,14 @@ fgfp8_status dispatch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, cons
   constexpr int kWideCW = 128;
   // UE8M0 scales: the tensor core applies them (block-scaled MMA), no promotion.
   if (fmt == FGFP8_SCALE_UE8M0)
-    return wide ? launch_gemm_mx<256, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms, early)
-                : launch_gemm_mx<128, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms, early);
+    return wide ? launch_gemm_mx<256, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms, early,
+                                                cap)
+                : launch_gemm_mx<128, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms, early,
+                                                cap);
   return wide ? launch_gemm<256, kWideCW, 0, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms,
-                                                       early)
+                                                       early, cap)
               : launch_gemm<128, 64, 0, kGrouped>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, offs, E, b_rows, s, dev, sms,
-                                                  early);
+                                                  early, cap);
 }
 
 // Few-token (M <= 64) launch: one CTA per 128 output columns, operands swapped.
@@ -683,6 +685,26 @@ fgfp8_status fgfp8_gemm_rowcol(const uint8_t* Xq, const float* sx, int x_per_ten
   return launch_gemm_rowcol<128>(Xq, sx, x_per_tensor, Wq, sw, w_per_tensor, Y, M, N, K, s, dev, info.sm_count);
 }
 
+fgfp8_status fgfp8_masked_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
+                               void* Y, const int32_t* counts, int32_t E, int64_t cap, int64_t N, int64_t K, int fmt,
+                               void* stream) {
+  if (E <= 0) return fail(FGFP8_ERR_INVALID_ARG, "E must be >= 1");
+  if (cap <= 0 || cap % 128 != 0) return fail(FGFP8_ERR_SHAPE, "cap must be a positive multiple of 128");
+  if (static_cast<int64_t>(E) * cap >= (int64_t(1) << 31)) return fail(FGFP8_ERR_SHAPE, "E*cap must be < 2^31");
+  const int64_t M_total = static_cast<int64_t>(E) * cap;
+  fgfp8_status st = check_gemm_common(Xq, Xs, ld_s, Wq, Ws, Y, M_total, N, K, fmt);
+  if (st != FGFP8_OK) return st;
+  if (!counts) return fail(FGFP8_ERR_INVALID_ARG, "counts is NULL");
+  if (!aligned(counts, 4)) return fail(FGFP8_ERR_ALIGN, "counts must be 4-byte aligned");
+  if (static_cast<int64_t>(E) * N >= (int64_t(1) << 31)) return fail(FGFP8_ERR_SHAPE, "E*N must be < 2^31");
+  int dev;
+  DeviceInfo info;
+  st = current_device(&dev, &info);
+  if (st != FGFP8_OK) return st;
+  return dispatch_gemm<true>(Xq, Xs, ld_s, Wq, Ws, Y, M_total, N, K, fmt, counts, E, static_cast<int64_t>(E) * N,
+                             reinterpret_cast<cudaStream_t>(stream), dev, info.sm_count, 0, static_cast<int>(cap));
+}
+
 fgfp8_status fgfp8_gemm_swiglu_quant(const uint8_t* Xq, const float* Xs, int64_t ld_s, const uint8_t* Wq_gu,
                                      const float* Ws_gu, uint8_t* Hq, float* Hs, int64_t ld_h, int64_t M, int64_t I,
                                      int64_t K, void* stream) {
@@ -698,8 +720,8 @@ fgfp8_status fgfp8_gemm_swiglu_quant(const uint8_t* Xq, const float* Xs, int64_t
   st = current_device(&dev, &info);
   if (st != FGFP8_OK) return st;
   return launch_gemm<256, 128, 0, false, true>(Xq, Xs, ld_s, Wq_gu, Ws_gu, nullptr, M, 2 * I, K, nullptr, 1, 2 * I,
-                                               reinterpret_cast<cudaStream_t>(stream), dev, info.sm_count, 0, Hq, Hs,
-                                               ld_h);
+                                               reinterpret_cast<cudaStream_t>(stream), dev, info.sm_count, 0, 0, Hq,
+                                               Hs, ld_h);
 }
 
 fgfp8_status fgfp8_check_device_status(void* stream) {

@@ -122,6 +122,22 @@ __device__ __forceinline__ int find_expert(const int32_t* __restrict__ offs, int
   return -1;
 }
 
+// Masked expert layout (cap > 0): expert e owns rows [e * cap, e * cap + cap);
+// its first counts[e] rows hold tokens and the rest are padding.  Returns the
+// expert of the M tile starting at row m0 (cap is a multiple of the tile
+// height, so a tile never straddles experts) and sets row_end to the end of
+// its token rows; -2 marks a tile of padding rows only (skipped, not an
+// error), -1 a count outside [0, cap] (skipped and recorded).
+__device__ __forceinline__ int masked_expert(const int32_t* __restrict__ counts, int E, int cap, int m0,
+                                             int& row_end) {
+  const int e = m0 / cap;
+  if (e >= E) return -1;
+  const int cnt = __ldg(counts + e);
+  if (cnt < 0 || cnt > cap) return -1;
+  row_end = e * cap + cnt;
+  return m0 < row_end ? e : -2;
+}
+
 // ---------------------------------------------------------------------------
 // Pipeline roles shared by the GEMM kernels.
 // ---------------------------------------------------------------------------
@@ -222,7 +238,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
     gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmBh, const void* __restrict__ Xs, uint32_t ld_s,
                             const void* __restrict__ Ws, __nv_bfloat16* __restrict__ Y, int M, int N, int K,
-                            const int32_t* __restrict__ group_offs, int E, int num_tiles, int num_full,
+                            const int32_t* __restrict__ group_offs, int E, int cap, int num_tiles, int num_full,
                             int early_b, uint8_t* __restrict__ Hq, float* __restrict__ Hs, uint32_t ld_h) {
   using C = GemmCfg<BN, CW>;
   static_assert(!kFuse || (BN == 256 && CW == 128 && FMT == 0 && !kGrouped), "fused SwiGLU: dense fp32 256-wide");
@@ -248,13 +264,18 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
   const int num_m = (M + C::kBM - 1) / C::kBM;
   const int num_n = N / BN;
 
-  // Work item t -> (m0, n0, expert, half).  Dense tiles run M-fastest (the
-  // activation tile set stays L2-resident while a weight tile is reused);
-  // grouped tiles run N-fastest (the CTAs of one expert share its weights in
-  // L2).  An expert of -1 marks a tile whose rows no segment covers: every
-  // role skips it and the status word records it.
-  auto coords = [&](int t, int& m0, int& n0, int& expert, bool& half) {
+  // Work item t -> (m0, n0, expert, half, row_end).  Dense tiles run
+  // M-fastest (the activation tile set stays L2-resident while a weight tile
+  // is reused); grouped tiles run N-fastest (the CTAs of one expert share its
+  // weights in L2).  Grouped rows come either as contiguous expert segments
+  // (group_offs, cap == 0) or in the masked layout (per-expert counts in
+  // group_offs, cap > 0).  An expert of -1 marks a tile whose rows no segment
+  // covers (every role skips it and the status word records it), -2 a
+  // masked tile of padding rows only (skipped).  Rows >= row_end of a tile
+  // are not stored.
+  auto coords = [&](int t, int& m0, int& n0, int& expert, bool& half, int& row_end) {
     half = false;
+    row_end = M;
     if (!kGrouped) {
       int f = t, h = 0;
       if (kHalfTiles && t >= num_full) {
@@ -268,7 +289,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
     } else {
       n0 = (t % num_n) * BN;
       m0 = (t / num_n) * C::kBM;
-      expert = find_expert(group_offs, E, m0);
+      expert = cap > 0 ? masked_expert(group_offs, E, cap, m0, row_end) : find_expert(group_offs, E, m0);
     }
   };
 
@@ -314,8 +335,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
       // written by the preceding grid).
       int pre = 0;
       bool half0 = true;
-      int m0p = 0, n0p = 0, ep = 0;
-      if (static_cast<int>(blockIdx.x) < num_tiles) coords(blockIdx.x, m0p, n0p, ep, half0);
+      int m0p = 0, n0p = 0, ep = 0, rep_end = 0;
+      if (static_cast<int>(blockIdx.x) < num_tiles) coords(blockIdx.x, m0p, n0p, ep, half0, rep_end);
       if (!kGrouped && early_b && static_cast<int>(blockIdx.x) < num_tiles && !half0) {
         const int n0 = n0p;
         pre = KB < C::kStages ? KB : C::kStages;
@@ -328,11 +349,11 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        int m0, n0, expert;
+        int m0, n0, expert, row_end;
         bool half;
-        coords(t, m0, n0, expert, half);
+        coords(t, m0, n0, expert, half, row_end);
         if (expert < 0) {
-          record_status(kDevBadGroupOffsets);
+          if (expert == -1) record_status(kDevBadGroupOffsets);
           continue;
         }
         const int b_row = expert * N + n0;
@@ -365,9 +386,9 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
       uint32_t it = 0, bt = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        int m0, n0, expert;
+        int m0, n0, expert, row_end;
         bool half;
-        coords(t, m0, n0, expert, half);
+        coords(t, m0, n0, expert, half, row_end);
         if (expert < 0) continue;
         const uint32_t idesc = (kHalfTiles && half) ? idesc_half : idesc_full;
         for (int kb = 0; kb < KB; ++kb, ++it, ++bt) {
@@ -422,11 +443,11 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
     // tile, CW/2 of a half tile; either way they lie in one 128-column
     // weight block.
     auto tile_rows = [&](int t, int& m0, int& n0, int& expert, bool& half, int& col0, int& m, bool& live,
-                         uint64_t& ws_row) {
-      coords(t, m0, n0, expert, half);
+                         uint64_t& ws_row, int& row_end) {
+      coords(t, m0, n0, expert, half, row_end);
       col0 = grp * ((kHalfTiles && half) ? CW / 2 : CW);
       m = m0 + row;
-      live = (m < M) && (n0 + col0 < N);
+      live = (m < row_end) && (n0 + col0 < N);
       ws_row = (static_cast<uint64_t>(expert < 0 ? 0 : expert) * NB + (n0 + col0) / 128) * KB;
     };
     int pref_t = -1;                           // tile whose first scale words are in the ring
@@ -527,7 +548,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
 
     // One work item with COLS columns per warp: per K block, the partial from
     // TMEM times sa * sw into the accumulators, then the bf16 epilogue.
-    auto promote = [&](auto cols_tag, int t, int m0, int n0, int col0, int m, bool live, uint64_t ws_row) {
+    auto promote = [&](auto cols_tag, int t, int m0, int n0, int col0, int m, bool live, uint64_t ws_row,
+                       int row_end) {
       constexpr int COLS = decltype(cols_tag)::value;
       const uint32_t lane_base =
           tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(col0);
@@ -581,10 +603,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
       pref_t = -1;
       if (t + static_cast<int>(gridDim.x) < num_tiles) {
         const int tn = t + static_cast<int>(gridDim.x);
-        int m0n, n0n, en, c0n, mn;
+        int m0n, n0n, en, c0n, mn, ren;
         bool hn, liven;
         uint64_t wsn;
-        tile_rows(tn, m0n, n0n, en, hn, c0n, mn, liven, wsn);
+        tile_rows(tn, m0n, n0n, en, hn, c0n, mn, liven, wsn, ren);
         if (en >= 0) {
 #pragma unroll
           for (int d = 0; d < kScaleAhead; ++d) fetch(d, mn, liven, wsn, ra[d], rw[d]);
@@ -627,17 +649,17 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
           const int r = 4 * i + (lane >> 3), c = lane & 7;
           const uint4 v = *reinterpret_cast<const uint4*>(slot + r * 128 + ((c ^ (r & 7)) << 4));
           const int mr = m0 + quad * 32 + r;
-          if (mr < M) *reinterpret_cast<uint4*>(Y + static_cast<uint64_t>(mr) * N + n0 + col0 + p * 64 + c * 8) = v;
+          if (mr < row_end) *reinterpret_cast<uint4*>(Y + static_cast<uint64_t>(mr) * N + n0 + col0 + p * 64 + c * 8) = v;
         }
         __syncwarp();
       }
     };
 
     for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-      int m0, n0, expert, col0, m;
+      int m0, n0, expert, col0, m, row_end;
       bool half, live;
       uint64_t ws_row;
-      tile_rows(t, m0, n0, expert, half, col0, m, live, ws_row);
+      tile_rows(t, m0, n0, expert, half, col0, m, live, ws_row, row_end);
       if (expert < 0) continue;
       if (pref_t != t) {
 #pragma unroll
@@ -645,11 +667,11 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
       }
       if constexpr (kHalfTiles) {
         if (half) {
-          promote(std::integral_constant<int, CW / 2>{}, t, m0, n0, col0, m, live, ws_row);
+          promote(std::integral_constant<int, CW / 2>{}, t, m0, n0, col0, m, live, ws_row, row_end);
           continue;
         }
       }
-      promote(std::integral_constant<int, CW>{}, t, m0, n0, col0, m, live, ws_row);
+      promote(std::integral_constant<int, CW>{}, t, m0, n0, col0, m, live, ws_row, row_end);
     }
   }
 
@@ -706,7 +728,7 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
     gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const uint8_t* __restrict__ Xs, uint32_t ld_s, const uint8_t* __restrict__ Ws,
                    __nv_bfloat16* __restrict__ Y, int M, int N, int K, const int32_t* __restrict__ group_offs,
-                   int E, int num_tiles, int early_b) {
+                   int E, int cap, int num_tiles, int early_b) {
   using C = MxCfg<BN>;
   static_assert(C::kSfCol + 2 * C::kSfColsPerKb <= C::kTmemCols, "TMEM columns");
   extern __shared__ uint8_t smem_raw[];
@@ -729,7 +751,10 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
   const int num_m = (M + C::kBM - 1) / C::kBM;
   const int num_n = N / C::kBN;
 
-  auto coords = [&](int t, int& m0, int& n0, int& expert) {
+  // as in the fp32-scale kernel: expert -1 = uncovered rows (recorded),
+  // -2 = masked padding tile (skipped); rows >= row_end are not stored
+  auto coords = [&](int t, int& m0, int& n0, int& expert, int& row_end) {
+    row_end = M;
     if (!kGrouped) {
       m0 = (t % num_m) * C::kBM;
       n0 = (t / num_m) * C::kBN;
@@ -737,7 +762,7 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
     } else {
       n0 = (t % num_n) * C::kBN;
       m0 = (t / num_n) * C::kBM;
-      expert = find_expert(group_offs, E, m0);
+      expert = cap > 0 ? masked_expert(group_offs, E, cap, m0, row_end) : find_expert(group_offs, E, m0);
     }
   };
 
@@ -777,8 +802,8 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
     // by the preceding grid).
     int pre = 0;
     if (!kGrouped && early_b && static_cast<int>(blockIdx.x) < num_tiles) {
-      int m0, n0, expert;
-      coords(blockIdx.x, m0, n0, expert);
+      int m0, n0, expert, row_end;
+      coords(blockIdx.x, m0, n0, expert, row_end);
       pre = KB < C::kStages ? KB : C::kStages;
       if (lane == 0) {
         for (int kb = 0; kb < pre; ++kb) {
@@ -791,10 +816,10 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
     uint32_t it = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-      int m0, n0, expert;
-      coords(t, m0, n0, expert);
+      int m0, n0, expert, row_end;
+      coords(t, m0, n0, expert, row_end);
       if (expert < 0) {
-        if (lane == 0) record_status(kDevBadGroupOffsets);
+        if (lane == 0 && expert == -1) record_status(kDevBadGroupOffsets);
         continue;
       }
       const uint64_t ws_row = (static_cast<uint64_t>(expert) * NB + n0 / 128) * KB;
@@ -805,7 +830,7 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int m = m0 + lane + 32 * j;
-          a[j] = (kb < KB && m < M) ? __ldg(Xs + static_cast<uint64_t>(kb) * ld_s + m) : 127u;
+          a[j] = (kb < KB && m < row_end) ? __ldg(Xs + static_cast<uint64_t>(kb) * ld_s + m) : 127u;
         }
 #pragma unroll
         for (int h = 0; h < BN / 128; ++h) w[h] = kb < KB ? __ldg(Ws + ws_row + static_cast<uint64_t>(h) * KB + kb) : 127u;
@@ -867,8 +892,8 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
       uint32_t it = 0, tile_no = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        int m0, n0, expert;
-        coords(t, m0, n0, expert);
+        int m0, n0, expert, row_end;
+        coords(t, m0, n0, expert, row_end);
         if (expert < 0) continue;
         const int ab = tile_no % C::kNumAcc;            // accumulator buffer
         const int tb = tile_no & 1;                      // tfull / tempty barrier of this tile
@@ -915,8 +940,8 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
     const int row = quad * 32 + lane;
     uint32_t tile_no = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-      int m0, n0, expert;
-      coords(t, m0, n0, expert);
+      int m0, n0, expert, row_end;
+      coords(t, m0, n0, expert, row_end);
       if (expert < 0) continue;
       const int ab = tile_no % C::kNumAcc;
       const int tb = tile_no & 1;
@@ -938,7 +963,7 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[tb]);
-      if (m < M) {
+      if (m < row_end) {
 #pragma unroll
         for (int j = 0; j < 128; j += 8) {
           uint4 v;

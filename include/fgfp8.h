@@ -140,6 +140,25 @@ fgfp8_status fgfp8_grouped_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s,
                                 int64_t M_total, int64_t N, int64_t K, int fmt, void* stream);
 
 /*
+ * Masked (batched) expert GEMM for decode-time MoE ("Fine-grained FP8",
+ * "DeepGEMM fast path": the experts backends, batched and masked expert
+ * layouts): every expert e owns a fixed block of cap rows, rows
+ * [e*cap, e*cap + cap), of which the first counts[e] hold tokens; rows
+ * [e*cap + counts[e], e*cap + cap) are padding that is never read into Y.
+ *   Xq, Xs, ld_s  as from fgfp8_quant_act over all E*cap rows (padding rows
+ *                 may hold anything).
+ *   Wq, Ws        [E, N, K] and [E, N/128, K/128] as for fgfp8_grouped_gemm.
+ *   Y             bf16 [E*cap, N]; only token rows are written.
+ *   counts        DEVICE int32 [E], each in [0, cap].
+ * cap % 128 == 0.  Tiles of padding rows only are skipped.  A count outside
+ * [0, cap] skips that expert's tiles and fgfp8_check_device_status then
+ * reports FGFP8_ERR_DEVICE.  Both scale formats are accepted.
+ */
+fgfp8_status fgfp8_masked_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
+                               void* Y, const int32_t* counts, int32_t E, int64_t cap, int64_t N, int64_t K, int fmt,
+                               void* stream);
+
+/*
  * The whole W8A8 linear layer: fgfp8_quant_act of X into the caller's Xq /
  * Xs buffers followed by fgfp8_gemm ("Fine-grained FP8", introduction and
  * "DeepGEMM fast path": activations are quantized on the fly, weights are

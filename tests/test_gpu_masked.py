@@ -1,0 +1,92 @@
+"""GPU parity of the masked (batched) expert GEMM: expert e's tokens occupy
+rows [e * cap, e * cap + counts[e]) of a fixed [E * cap, K] buffer, the rest
+is padding.  Token rows against the oracle (per expert, its own weights);
+padding rows of Y never written; with every expert full the result equals the
+contiguous grouped GEMM; an out-of-range count is reported without a fault."""
+import numpy as np
+import pytest
+import torch
+
+import fine_grained_fp8_token_b200 as fg
+import oracle
+import workloads
+from parity import F32, UE8M0, assert_gemm_close, bits16, require_gpu, to_np, y_to_f64
+
+pytestmark = pytest.mark.gpu
+SENTINEL = 7.0
+
+
+@pytest.fixture(scope="module")
+def dev():
+    d = require_gpu()
+    fg.load()
+    return d
+
+
+def build(dev, E, cap, N, K, fmt, seed, nan_padding=True, counts=None):
+    X = workloads.activations((E * cap, K), "normal_outliers", seed=seed)
+    if nan_padding and counts is not None:
+        for e, c in enumerate(counts):
+            if c < cap:
+                X[e * cap + c:(e + 1) * cap, ::7] = float("nan")     # padding may hold anything
+    Wq = torch.empty((E, N, K), dtype=torch.uint8, device=dev)
+    Ws = torch.empty((E, N // 128, K // 128), dtype=torch.float32 if fmt == F32 else torch.uint8, device=dev)
+    W_list = []
+    for e in range(E):
+        W = workloads.weights((N, K), seed=seed + 1 + e)
+        W_list.append(W)
+        fg.quant_weight(W.to(dev), fmt, Wq=Wq[e], Ws=Ws[e])
+    Xq, Xs = fg.quant_act(X.to(dev), fmt)
+    return X, W_list, Xq, Xs, Wq, Ws
+
+
+def check_rows(X, W_list, Y, counts, cap, fmt, what):
+    for e, c in enumerate(counts):
+        if c == 0:
+            continue
+        rows = slice(e * cap, e * cap + c)
+        Xq_r, Xs_r = oracle.quant_act(bits16(X[rows]), fmt)
+        Wq_r, Ws_r = oracle.quant_weight(bits16(W_list[e]), fmt)
+        Y_ref, S = oracle.gemm(Xq_r, Xs_r, Wq_r, Ws_r, fmt)
+        assert_gemm_close(y_to_f64(Y[rows]), Y_ref, S, f"{what} expert {e}")
+
+
+@pytest.mark.parametrize("fmt", [F32, UE8M0])
+@pytest.mark.parametrize("cap,counts,N", [(128, [0, 3, 128, 77, 1], 256), (256, [256, 130, 0, 200], 384)])
+def test_masked_gemm(dev, fmt, cap, counts, N):
+    E, K = len(counts), 512
+    X, W_list, Xq, Xs, Wq, Ws = build(dev, E, cap, N, K, fmt, seed=cap + N + fmt, counts=counts)
+    cnt = torch.tensor(counts, dtype=torch.int32, device=dev)
+    Y = torch.full((E * cap, N), SENTINEL, dtype=torch.bfloat16, device=dev)
+    fg.masked_gemm(Xq, Xs, Wq, Ws, cnt, fmt, Y=Y)
+    fg.check_device_status()
+    check_rows(X, W_list, Y, counts, cap, fmt, f"masked cap {cap}")
+    for e, c in enumerate(counts):
+        assert (Y[e * cap + c:(e + 1) * cap].float() == SENTINEL).all(), f"padding rows of expert {e} written"
+
+
+@pytest.mark.parametrize("fmt", [F32, UE8M0])
+def test_masked_full_equals_grouped(dev, fmt):
+    E, cap, N, K = 3, 256, 256, 1024
+    X, W_list, Xq, Xs, Wq, Ws = build(dev, E, cap, N, K, fmt, seed=41, nan_padding=False)
+    cnt = torch.full((E,), cap, dtype=torch.int32, device=dev)
+    Y_m = fg.masked_gemm(Xq, Xs, Wq, Ws, cnt, fmt)
+    offs = torch.arange(0, (E + 1) * cap, cap, dtype=torch.int32, device=dev)
+    Y_g = fg.grouped_gemm(Xq, Xs, Wq, Ws, offs, fmt)
+    fg.check_device_status()
+    assert torch.equal(Y_m, Y_g)
+
+
+def test_masked_bad_count_reported(dev):
+    E, cap, N, K = 3, 128, 256, 256
+    counts = [5, cap + 1, 128]
+    X, W_list, Xq, Xs, Wq, Ws = build(dev, E, cap, N, K, F32, seed=7, counts=[5, cap, 128])
+    cnt = torch.tensor(counts, dtype=torch.int32, device=dev)
+    Y = torch.full((E * cap, N), SENTINEL, dtype=torch.bfloat16, device=dev)
+    fg.masked_gemm(Xq, Xs, Wq, Ws, cnt, F32, Y=Y)
+    with pytest.raises(fg.FGFP8Error) as ei:
+        fg.check_device_status()
+    assert ei.value.status == 7
+    assert (Y[cap:2 * cap].float() == SENTINEL).all()          # the bad expert's rows untouched
+    check_rows(X, W_list, Y, [5, 0, 128], cap, F32, "bad-count neighbours")
+    fg.check_device_status()                                    # cleared

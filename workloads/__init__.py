@@ -66,6 +66,9 @@ MOE = MoE("deepseek_v3_moe_256x4096x7168_top8")
 # the same expert shapes with 32 experts and 512 tokens (~1 GB of weights): a
 # profiling case larger than L2 but small enough for multi-pass captures
 MOE_SMALL = MoE("deepseek_v3_moe_32x4096x7168_top8_512tok", E=32, tokens=512)
+# decode step of the same expert layer: 128 tokens, top-8, in the masked
+# layout (every expert a fixed block of 128 rows, its first counts[e] used)
+MOE_DECODE = MoE("deepseek_v3_moe_decode_masked_256x4096x7168_top8_128tok", tokens=128)
 
 LINEARS = {c.name: c for c in [TINY, LLAMA_ATTN, LLAMA_GATE_UP, LLAMA_DOWN, *DS_DECODE.values()]}
 
@@ -159,6 +162,18 @@ def moe_grouped_rows(X_tok: torch.Tensor, routing: Routing) -> torch.Tensor:
     X = torch.zeros((routing.M_total, X_tok.shape[1]), dtype=X_tok.dtype, device=X_tok.device)
     valid = idx >= 0
     X[valid] = X_tok[idx[valid]]
+    return X
+
+
+def moe_masked_rows(X_tok: torch.Tensor, routing: Routing, E: int, cap: int) -> torch.Tensor:
+    """X [E * cap, K] in the masked layout: expert e's routed tokens (in
+    ascending token order) in rows [e * cap, e * cap + counts[e]), zeros in
+    the rest of its block."""
+    X = torch.zeros((E * cap, X_tok.shape[1]), dtype=X_tok.dtype, device=X_tok.device)
+    for e in range(E):
+        seg = routing.row_token[routing.group_offs[e]:routing.group_offs[e] + routing.counts[e]]
+        if len(seg):
+            X[e * cap:e * cap + len(seg)] = X_tok[torch.as_tensor(seg, device=X_tok.device)]
     return X
 
 
