@@ -71,6 +71,7 @@ WORKLOAD_ALIASES = {
     "llama_down_dynamic": f"{workloads.LLAMA_DOWN.name}_fp8_dynamic",
     "llama_mlp_fused": "llama3_8b_mlp_8192x4096x14336_swiglu_fused",
     "moe_decode_masked": workloads.MOE_DECODE.name,
+    "moe_decode_masked_small": workloads.MOE_DECODE_SMALL.name,
 }
 MLP_NAME = "llama3_8b_mlp_8192x4096x14336_swiglu_fused"
 
@@ -328,9 +329,11 @@ class MLPLayer:
     M, K, I, N_DOWN = 8192, 4096, 14336, 4096
     launches_per_step = 3
 
-    def __init__(self, dev):
+    def __init__(self, dev, tokens=None):
         import fine_grained_fp8_token_b200 as fg
         self.fg, self.dev = fg, dev
+        if tokens:
+            self.M = tokens                 # a smaller token batch of the same layer (profiling captures)
         c = workloads.LLAMA_GATE_UP
         self.X = workloads.activations((self.M, self.K), c.x_kind, c.seed, device=dev)
         Wg = workloads.weights((self.I, self.K), c.seed + 1, device=dev)
@@ -382,7 +385,8 @@ class MLPLayer:
         return 3.0 * 2 * self.I * self.K + 4.0 * 2 * self.I * self.K / 16384
 
     def describe(self):
-        return {"workload": MLP_NAME, "M": self.M, "K": self.K, "I": self.I, "N_down": self.N_DOWN,
+        return {"workload": MLP_NAME if self.M == MLPLayer.M else f"{MLP_NAME}@{self.M}tok", "M": self.M,
+                "K": self.K, "I": self.I, "N_down": self.N_DOWN,
                 "scales": "fp32 (1x128 activations, 128x128 weights)", "x": "normal_outliers",
                 "chain": "quant_act -> gate/up GEMM + SiLU*up + quant (fused) -> down GEMM"}
 
@@ -536,12 +540,13 @@ class MoELayer:
         return ("gemm_blockscaled_kernel" if self.cfg.fmt == 0 else "gemm_mx_kernel") + " (grouped)"
 
 
-def make_layer(name, dev):
+def make_layer(name, dev, tokens=None):
     name = WORKLOAD_ALIASES.get(name, name)
-    if name == workloads.MOE_DECODE.name:
-        return MaskedMoELayer(workloads.MOE_DECODE, dev)
+    for cfg in (workloads.MOE_DECODE, workloads.MOE_DECODE_SMALL):
+        if name == cfg.name:
+            return MaskedMoELayer(cfg, dev)
     if name == MLP_NAME:
-        return MLPLayer(dev)
+        return MLPLayer(dev, tokens)
     if name in ROWCOL:
         cfg, scheme = ROWCOL[name]
         return RowColLayer(cfg, scheme, dev)
@@ -576,7 +581,7 @@ def run_gpu(args, rank, world, dev):
     programmatic dependent), bracketed by CUDA events; a second pass of the
     same length times the two kernels apart (an event between them) for the
     per-kernel roofline."""
-    layer = make_layer(args.workload, dev)
+    layer = make_layer(args.workload, dev, args.tokens)
     stream = torch.cuda.current_stream(dev)
     flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
@@ -712,9 +717,10 @@ class OracleSample:
             self.desc = (f"first {self.rows} of {cfg.M} rows x the full [{cfg.N}, {cfg.K}] weight, "
                          f"{self.scheme} scales")
             return
-        if name in (workloads.MOE.name, workloads.MOE_SMALL.name, workloads.MOE_DECODE.name):
-            cfg = {workloads.MOE.name: workloads.MOE, workloads.MOE_SMALL.name: workloads.MOE_SMALL,
-                   workloads.MOE_DECODE.name: workloads.MOE_DECODE}[name]
+        moe = {c.name: c for c in (workloads.MOE, workloads.MOE_SMALL, workloads.MOE_DECODE,
+                                   workloads.MOE_DECODE_SMALL)}
+        if name in moe:
+            cfg = moe[name]
             r = workloads.moe_routing(cfg)
             e = int(np.argmax(r.counts))                    # the busiest expert's rows
             tok = r.row_token[r.group_offs[e]:r.group_offs[e] + r.counts[e]]
@@ -830,6 +836,8 @@ def main():
                     help="one of: " + ", ".join(WORKLOAD_ALIASES))
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (quick runs)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="token batch of the fused MLP workload (default: its 8192; smaller for profiling captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -69,6 +69,7 @@ MOE_SMALL = MoE("deepseek_v3_moe_32x4096x7168_top8_512tok", E=32, tokens=512)
 # decode step of the same expert layer: 128 tokens, top-8, in the masked
 # layout (every expert a fixed block of 128 rows, its first counts[e] used)
 MOE_DECODE = MoE("deepseek_v3_moe_decode_masked_256x4096x7168_top8_128tok", tokens=128)
+MOE_DECODE_SMALL = MoE("deepseek_v3_moe_decode_masked_32x4096x7168_top8_64tok", E=32, tokens=64)
 
 LINEARS = {c.name: c for c in [TINY, LLAMA_ATTN, LLAMA_GATE_UP, LLAMA_DOWN, *DS_DECODE.values()]}
 
