@@ -293,11 +293,14 @@ fgfp8_status launch_gemm_rowcol(const uint8_t* Xq, const float* sx, int x_per_te
                                 const float* sw, int w_per_tensor, void* Y, int64_t M, int64_t N, int64_t K,
                                 cudaStream_t stream, int dev, int sm_count) {
   using C = fgfp8::RowColCfg<BN>;
-  CUtensorMap mA, mB;
+  CUtensorMap mA, mB, mBh;
   fgfp8_status st = make_map_u8_sw128(&mA, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
                                       static_cast<uint64_t>(K), 128);
   if (st != FGFP8_OK) return st;
   st = make_map_u8_sw128(&mB, Wq, static_cast<uint64_t>(N), static_cast<uint64_t>(K), static_cast<uint64_t>(K), BN);
+  if (st != FGFP8_OK) return st;
+  st = make_map_u8_sw128(&mBh, Wq, static_cast<uint64_t>(N), static_cast<uint64_t>(K), static_cast<uint64_t>(K),
+                         BN / 2);
   if (st != FGFP8_OK) return st;
   auto kernel = fgfp8::gemm_rowcol_kernel<BN>;
   st = set_smem(reinterpret_cast<const void*>(kernel), C::kSmemBytes, dev);
@@ -305,10 +308,19 @@ fgfp8_status launch_gemm_rowcol(const uint8_t* Xq, const float* sx, int x_per_te
   const int64_t tiles = ((M + C::kBM - 1) / C::kBM) * (N / BN);
   if (tiles == 0) return ok();
   const int64_t grid = tiles < sm_count ? tiles : sm_count;
+  // the last partial wave as half tiles when it fits twice into one wave
+  int64_t num_full = tiles, items = tiles;
+  if (BN == 256) {
+    const int64_t waves = tiles / grid, rest = tiles - waves * grid;
+    if (waves >= 1 && rest > 0 && 2 * rest <= grid) {
+      num_full = waves * grid;
+      items = num_full + 2 * rest;
+    }
+  }
   return launch_dependent(kernel, static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, stream,
-                          "row/column-scaled gemm launch", mA, mB, sx, x_per_tensor, sw, w_per_tensor,
+                          "row/column-scaled gemm launch", mA, mB, mBh, sx, x_per_tensor, sw, w_per_tensor,
                           reinterpret_cast<__nv_bfloat16*>(Y), static_cast<int>(M), static_cast<int>(N),
-                          static_cast<int>(K), static_cast<int>(tiles));
+                          static_cast<int>(K), static_cast<int>(items), static_cast<int>(num_full));
 }
 
 // Shared checks of the row / tensor quantizers' input X bf16 [R, K] (row
@@ -608,9 +620,14 @@ fgfp8_status fgfp8_quant_rows(const void* X, int64_t R, int64_t K, int64_t ldx, 
   DeviceInfo info;
   st = current_device(&dev, &info);
   if (st != FGFP8_OK) return st;
-  fgfp8::quant_rows_kernel<<<static_cast<unsigned>(R), fgfp8::kRowThreads, 0,
-                             reinterpret_cast<cudaStream_t>(stream)>>>(
-      reinterpret_cast<const uint16_t*>(X), static_cast<uint32_t>(K), static_cast<uint64_t>(ldx), Xq, scales);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (K <= fgfp8::kWarpRowChunks * 32 * 8)
+    fgfp8::quant_rows_warp_kernel<<<static_cast<unsigned>((R + 7) / 8), 256, 0, s>>>(
+        reinterpret_cast<const uint16_t*>(X), static_cast<uint32_t>(R), static_cast<uint32_t>(K),
+        static_cast<uint64_t>(ldx), Xq, scales);
+  else
+    fgfp8::quant_rows_kernel<<<static_cast<unsigned>(R), fgfp8::kRowThreads, 0, s>>>(
+        reinterpret_cast<const uint16_t*>(X), static_cast<uint32_t>(K), static_cast<uint64_t>(ldx), Xq, scales);
   return check_launch("quant_rows launch");
 }
 

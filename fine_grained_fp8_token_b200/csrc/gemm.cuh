@@ -1023,9 +1023,11 @@ struct RowColCfg {
 template <int BN>
 __global__ void __launch_bounds__(RowColCfg<BN>::kThreads, 1)
     gemm_rowcol_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                       const float* __restrict__ sx, int x_per_tensor, const float* __restrict__ sw,
-                       int w_per_tensor, __nv_bfloat16* __restrict__ Y, int M, int N, int K, int num_tiles) {
+                       const __grid_constant__ CUtensorMap tmBh, const float* __restrict__ sx, int x_per_tensor,
+                       const float* __restrict__ sw, int w_per_tensor, __nv_bfloat16* __restrict__ Y, int M, int N,
+                       int K, int num_tiles, int num_full) {
   using C = RowColCfg<BN>;
+  constexpr bool kHalfTiles = BN == 256;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -1041,10 +1043,18 @@ __global__ void __launch_bounds__(RowColCfg<BN>::kThreads, 1)
   const int lane = threadIdx.x & 31;
   const int KB = K / C::kBK;
   const int num_m = (M + C::kBM - 1) / C::kBM;
-  // tile t -> (m0, n0), M-fastest
-  auto coords = [&](int t, int& m0, int& n0) {
-    m0 = (t % num_m) * C::kBM;
-    n0 = (t / num_m) * C::kBN;
+  // work item t -> (m0, n0, half), M-fastest; items t >= num_full are the
+  // 128 x 128 halves of the remaining full tiles (as in the fp32-scale kernel)
+  auto coords = [&](int t, int& m0, int& n0, bool& half) {
+    int f = t, h = 0;
+    half = false;
+    if (kHalfTiles && t >= num_full) {
+      f = num_full + ((t - num_full) >> 1);
+      h = (t - num_full) & 1;
+      half = true;
+    }
+    m0 = (f % num_m) * C::kBM;
+    n0 = (f / num_m) * C::kBN + h * (C::kBN / 2);
   };
 
   if (threadIdx.x == 0) {
@@ -1062,6 +1072,7 @@ __global__ void __launch_bounds__(RowColCfg<BN>::kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (kHalfTiles) tma_prefetch_desc(&tmBh);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::kTmemCols);
@@ -1081,7 +1092,10 @@ __global__ void __launch_bounds__(RowColCfg<BN>::kThreads, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         int m0, n0;
-        coords(t, m0, n0);
+        bool half;
+        coords(t, m0, n0, half);
+        const CUtensorMap* mapB = (kHalfTiles && half) ? &tmBh : &tmB;
+        const uint32_t stage_tx = (kHalfTiles && half) ? C::kABytes + C::kBBytes / 2 : C::kStageBytes;
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % C::kStages;
           if (it >= static_cast<uint32_t>(C::kStages) && !mbar_wait(&empty[s], ((it / C::kStages) & 1u) ^ 1u)) {
@@ -1089,8 +1103,8 @@ __global__ void __launch_bounds__(RowColCfg<BN>::kThreads, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-          tma_load_2d(sB + s * C::kBBytes, &tmB, &full[s], kb * C::kBK, n0);
+          mbar_arrive_expect_tx(&full[s], stage_tx);
+          tma_load_2d(sB + s * C::kBBytes, mapB, &full[s], kb * C::kBK, n0);
           tma_load_2d(sA + s * C::kABytes, &tmA, &full[s], kb * C::kBK, m0);
         }
       }
@@ -1101,11 +1115,16 @@ __global__ void __launch_bounds__(RowColCfg<BN>::kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ================= MMA issuer
-      constexpr uint32_t idesc = idesc_e4m3_f32(128, C::kBN);
+      constexpr uint32_t idesc_full = idesc_e4m3_f32(128, C::kBN);
+      constexpr uint32_t idesc_half = idesc_e4m3_f32(128, C::kBN / 2);
       const uint64_t a_desc0 = smem_desc_k_sw128(smem_u32(sA)), b_desc0 = smem_desc_k_sw128(smem_u32(sB));
       uint32_t it = 0, tile_no = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++tile_no) {
+        int m0, n0;
+        bool half;
+        coords(t, m0, n0, half);
+        const uint32_t idesc = (kHalfTiles && half) ? idesc_half : idesc_full;
         const int ab = tile_no & 1;                      // accumulator and its tfull / tempty barriers
         if (tile_no >= 2 && !mbar_wait(&tempty[ab], ((tile_no - 2) >> 1) & 1u)) {
           record_status(kDevTimeoutMma);
@@ -1143,13 +1162,21 @@ __global__ void __launch_bounds__(RowColCfg<BN>::kThreads, 1)
     uint32_t tile_no = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++tile_no) {
       int m0, n0;
-      coords(t, m0, n0);
+      bool half;
+      coords(t, m0, n0, half);
       const int ab = tile_no & 1;
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[ab], (tile_no >> 1) & 1u))) {
         if (lane == 0) record_status(kDevTimeoutEpilogue);
         break;
       }
       tc_fence_after();
+      if (kHalfTiles && half && col0 >= C::kBN / 2) {
+        // no columns of this half tile: hand the accumulator back at once
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[ab]);
+        continue;
+      }
       const int m = m0 + row;
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(ab * C::kBN + col0);

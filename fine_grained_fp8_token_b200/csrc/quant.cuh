@@ -288,6 +288,42 @@ __global__ void __launch_bounds__(kRowThreads) quant_rows_kernel(const uint16_t*
   if (threadIdx.x == 0) scales[r] = gs.s;
 }
 
+// Rows of up to kWarpRowChunks * 32 * 8 = 4096 elements: one warp per row,
+// eight rows per CTA, every chunk held in registers between the warp's amax
+// reduction and the codes.  Same arithmetic as quant_rows_kernel.
+constexpr int kWarpRowChunks = 16;
+
+__global__ void __launch_bounds__(256) quant_rows_warp_kernel(const uint16_t* __restrict__ X, uint32_t R,
+                                                              uint32_t K, uint64_t ldx, uint8_t* __restrict__ Xq,
+                                                              float* __restrict__ scales) {
+  griddep_launch_dependents();
+  const uint32_t r = blockIdx.x * 8u + (threadIdx.x >> 5);
+  const uint32_t lane = threadIdx.x & 31u;
+  if (r >= R) return;
+  const uint16_t* xr = X + static_cast<uint64_t>(r) * ldx;
+  uint8_t* qr = Xq + static_cast<uint64_t>(r) * K;
+  const uint32_t chunks = K / 8;
+  uint4 v[kWarpRowChunks];
+  uint32_t a = 0;
+#pragma unroll
+  for (int i = 0; i < kWarpRowChunks; ++i) {
+    const uint32_t c = lane + i * 32u;
+    if (c < chunks) {
+      v[i] = ld_stream_v4(xr + c * 8u);
+      a = max(a, absmax_bits8(v[i]));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = max(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+  const GroupScale gs = make_scale<0>(a);
+#pragma unroll
+  for (int i = 0; i < kWarpRowChunks; ++i) {
+    const uint32_t c = lane + i * 32u;
+    if (c < chunks) *reinterpret_cast<uint2*>(qr + c * 8u) = quant8<0>(v[i], gs);
+  }
+  if (lane == 0) scales[r] = gs.s;
+}
+
 // amax over a whole tensor: each thread folds 16-byte chunks of its
 // grid-stride share, the warp reduces, lane 0 raises *amax_bits (bf16
 // magnitude bits; NaN patterns order above infinity) with atomicMax.
