@@ -72,6 +72,9 @@ WORKLOAD_ALIASES = {
     "llama_mlp_fused": "llama3_8b_mlp_8192x4096x14336_swiglu_fused",
     "moe_decode_masked": workloads.MOE_DECODE.name,
     "moe_decode_masked_small": workloads.MOE_DECODE_SMALL.name,
+    **{f"{a}_ue8m0": workloads.LLAMA_UE8M0[c.name].name
+       for a, c in (("llama_attn", workloads.LLAMA_ATTN), ("llama_gate_up", workloads.LLAMA_GATE_UP),
+                    ("llama_down", workloads.LLAMA_DOWN))},
 }
 MLP_NAME = "llama3_8b_mlp_8192x4096x14336_swiglu_fused"
 

@@ -215,12 +215,15 @@ fgfp8_status launch_gemm_mx(const uint8_t* Xq, const void* Xs, int64_t ld_s, con
                             void* Y, int64_t M, int64_t N, int64_t K, const int32_t* offs, int E, int64_t b_rows,
                             cudaStream_t stream, int dev, int sm_count, int early, int cap) {
   using C = fgfp8::MxCfg<BN>;
-  CUtensorMap mA, mB;
+  CUtensorMap mA, mB, mBh;
   fgfp8_status st = make_map_u8_sw128(&mA, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
                                       static_cast<uint64_t>(K), 128);
   if (st != FGFP8_OK) return st;
   st = make_map_u8_sw128(&mB, Wq, static_cast<uint64_t>(b_rows), static_cast<uint64_t>(K), static_cast<uint64_t>(K),
                          C::kBN);
+  if (st != FGFP8_OK) return st;
+  st = make_map_u8_sw128(&mBh, Wq, static_cast<uint64_t>(b_rows), static_cast<uint64_t>(K), static_cast<uint64_t>(K),
+                         C::kBN / 2);
   if (st != FGFP8_OK) return st;
   auto kernel = fgfp8::gemm_mx_kernel<BN, kGrouped>;
   st = set_smem(reinterpret_cast<const void*>(kernel), C::kSmemBytes, dev);
@@ -228,11 +231,22 @@ fgfp8_status launch_gemm_mx(const uint8_t* Xq, const void* Xs, int64_t ld_s, con
   const int64_t tiles = ((M + C::kBM - 1) / C::kBM) * (N / C::kBN);
   if (tiles == 0) return ok();
   const int64_t grid = tiles < sm_count ? tiles : sm_count;
+  // dense 128 x 256 tiles: the last partial wave as half tiles when it fits
+  // twice into one wave
+  int64_t num_full = tiles, items = tiles;
+  if (!kGrouped && BN == 256) {
+    const int64_t waves = tiles / grid, rest = tiles - waves * grid;
+    if (waves >= 1 && rest > 0 && 2 * rest <= grid) {
+      num_full = waves * grid;
+      items = num_full + 2 * rest;
+    }
+  }
   return launch_dependent(kernel, static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, stream,
-                          "block-scaled gemm launch", mA, mB, reinterpret_cast<const uint8_t*>(Xs),
+                          "block-scaled gemm launch", mA, mB, mBh, reinterpret_cast<const uint8_t*>(Xs),
                           static_cast<uint32_t>(ld_s), reinterpret_cast<const uint8_t*>(Ws),
                           reinterpret_cast<__nv_bfloat16*>(Y), static_cast<int>(M), static_cast<int>(N),
-                          static_cast<int>(K), offs, E, cap, static_cast<int>(tiles), early);
+                          static_cast<int>(K), offs, E, cap, static_cast<int>(items), static_cast<int>(num_full),
+                          early);
 }
 
 template <bool kGrouped>

@@ -689,18 +689,26 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
 // (the 128x128 weight block's scale, shared by its 128 rows) from TMEM
 // (kind::mxf8f6f4.block_scale, one scale per 32-element K slice; the four
 // slices of a 128 block use the same scale), so the whole K reduction
-// accumulates in TMEM and no promotion step runs per K block.
-//   warp 0      TMA for the operand tiles (lane 0) and, with all 32 lanes,
-//               the scale rows of each K block written to shared memory in
-//               the TMEM scale layout (lane l: scales of rows l, l+32, l+64,
-//               l+96, each byte repeated for the four K slices);
-//   warp 1      owns TMEM: per K block tcgen05.cp of the two scale tiles
-//               into TMEM, then four block-scaled MMAs; after the tile's last
-//               K block it publishes the accumulator (two buffers, so the
-//               epilogue of one tile overlaps the MMAs of the next);
-//   warps 4..7  epilogue: TMEM -> registers -> bf16 -> global.
-// TMEM: accumulators in columns [0, 256) (2 x 128), scale factors in
-// [256, 272) (2 K-block parities x (4 columns for A + 4 for B)).
+// accumulates in TMEM and no promotion step runs per K block.  The scales
+// travel in groups of four K blocks: byte b of each 32-bit TMEM scale word
+// belongs to K block 4g + b, and the MMAs of that block select it through
+// the scale-factor ids of the instruction descriptor, so one copy into TMEM
+// serves four K blocks.
+//   warp 0      TMA for the operand tiles (lane 0);
+//   warp 1      owns TMEM; per scale group tcgen05.cp of the group's slot
+//               into TMEM, then per K block four block-scaled MMAs; after the
+//               tile's last K block it publishes the accumulator.  The copies
+//               stay on this thread: the tensor pipe runs them in issue order
+//               with the MMAs, so no wait separates a copy from its MMAs;
+//   warp 2      the scale words of two groups at a time written to
+//               shared-memory slots in the TMEM scale layout (lane l: words
+//               of rows l, l+32, l+64, l+96; a weight tile: its block's word
+//               everywhere), one proxy fence per two groups, so the scale
+//               loads never delay a TMA or MMA issue;
+//   warps 4..   epilogue: TMEM -> registers -> bf16 -> global.
+// TMEM: BN = 128: two accumulators in columns [0, 256); BN = 256: one in
+// [0, 256).  Scale factors follow, two slots of 4 columns for A and BN / 32
+// for B.
 // ---------------------------------------------------------------------------
 template <int BN>
 struct MxCfg {
@@ -714,35 +722,42 @@ struct MxCfg {
   static constexpr uint32_t kSfBBytes = 512 * (BN / 128);         // one 32 x 16 tile per 128 rows of B
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;      // TMA bytes per stage
   static constexpr int kStages = (BN == 128) ? 6 : 4;
+  static constexpr int kSfGroup = 4;                              // K blocks per scale group (bytes of a word)
+  static constexpr int kSfBatch = 2;                              // groups written per shared-memory fence
+  static constexpr int kSfSlots = 2 * kSfBatch;                   // scale groups in flight
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kSfCol = kNumAcc * BN;                // scale factors after the accumulators
-  static constexpr uint32_t kSfColsPerKb = 4 + BN / 32;           // A: 4 columns, B: BN/32 columns
+  static constexpr uint32_t kSfColsPerSlot = 4 + BN / 32;         // A: 4 columns, B: BN/32 columns
   static constexpr size_t kBarrierBytes = 256;
-  static constexpr size_t kSmemBytes =
-      1024 + kStages * static_cast<size_t>(kStageBytes + kSfABytes + kSfBBytes) + kBarrierBytes;
-  static constexpr int kPrefetch = 4;                             // scale prefetch depth (K blocks)
+  static constexpr size_t kSmemBytes = 1024 + kStages * static_cast<size_t>(kStageBytes) +
+                                       kSfSlots * static_cast<size_t>(kSfABytes + kSfBBytes) + kBarrierBytes;
 };
 
 template <int BN, bool kGrouped>
 __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
     gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const uint8_t* __restrict__ Xs, uint32_t ld_s, const uint8_t* __restrict__ Ws,
-                   __nv_bfloat16* __restrict__ Y, int M, int N, int K, const int32_t* __restrict__ group_offs,
-                   int E, int cap, int num_tiles, int early_b) {
+                   const __grid_constant__ CUtensorMap tmBh, const uint8_t* __restrict__ Xs, uint32_t ld_s,
+                   const uint8_t* __restrict__ Ws, __nv_bfloat16* __restrict__ Y, int M, int N, int K,
+                   const int32_t* __restrict__ group_offs, int E, int cap, int num_tiles, int num_full,
+                   int early_b) {
   using C = MxCfg<BN>;
-  static_assert(C::kSfCol + 2 * C::kSfColsPerKb <= C::kTmemCols, "TMEM columns");
+  constexpr bool kHalfTiles = !kGrouped && BN == 256;
+  static_assert(C::kSfCol + C::kSfSlots * C::kSfColsPerSlot <= C::kTmemCols, "TMEM columns");
+  static_assert((2 * C::kStages + 4 + 1 + 2 * C::kSfSlots) * 8 + 4 <= C::kBarrierBytes, "barrier area");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = sA + C::kStages * C::kABytes;
   uint8_t* sSfA = sB + C::kStages * C::kBBytes;
-  uint8_t* sSfB = sSfA + C::kStages * C::kSfABytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sSfB + C::kStages * C::kSfBBytes);
+  uint8_t* sSfB = sSfA + C::kSfSlots * C::kSfABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sSfB + C::kSfSlots * C::kSfBBytes);
   uint64_t* empty = full + C::kStages;
   uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* mma_done = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* sf_full = mma_done + 1;                  // a scale group written to its shared-memory slot
+  uint64_t* sf_empty = sf_full + C::kSfSlots;        // the slot copied into TMEM
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_empty + C::kSfSlots);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -752,12 +767,21 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
   const int num_n = N / C::kBN;
 
   // as in the fp32-scale kernel: expert -1 = uncovered rows (recorded),
-  // -2 = masked padding tile (skipped); rows >= row_end are not stored
-  auto coords = [&](int t, int& m0, int& n0, int& expert, int& row_end) {
+  // -2 = masked padding tile (skipped); rows >= row_end are not stored;
+  // dense work items t >= num_full are 128 x 128 halves of the last full
+  // tiles (half = true: a 128-row weight box, an N = 128 MMA)
+  auto coords = [&](int t, int& m0, int& n0, int& expert, int& row_end, bool& half) {
     row_end = M;
+    half = false;
     if (!kGrouped) {
-      m0 = (t % num_m) * C::kBM;
-      n0 = (t / num_m) * C::kBN;
+      int f = t, h = 0;
+      if (kHalfTiles && t >= num_full) {
+        f = num_full + ((t - num_full) >> 1);
+        h = (t - num_full) & 1;
+        half = true;
+      }
+      m0 = (f % num_m) * C::kBM;
+      n0 = (f / num_m) * C::kBN + h * (C::kBN / 2);
       expert = 0;
     } else {
       n0 = (t % num_n) * C::kBN;
@@ -768,12 +792,16 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full[s], 2);                  // TMA bytes (+1 arrival) and the scale rows (+1 arrival)
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], C::kEpiWarps);
+    }
+    for (int b = 0; b < C::kSfSlots; ++b) {
+      mbar_init(&sf_full[b], 1);
+      mbar_init(&sf_empty[b], 1);
     }
     mbar_init(mma_done, 1);
     fence_mbarrier_init();
@@ -781,6 +809,7 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (kHalfTiles) tma_prefetch_desc(&tmBh);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::kTmemCols);
@@ -796,105 +825,152 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
   if (warp != 0) griddep_wait();
 
   if (warp == 0) {
-    // ================= producer: TMA (lane 0) + scale rows (all lanes)
+    // ================= producer: TMA (lane 0)
     // early_b (dense): the weight tiles of the first tile's first kStages K
     // blocks are requested before the wait (the weights must not be written
     // by the preceding grid).
-    int pre = 0;
-    if (!kGrouped && early_b && static_cast<int>(blockIdx.x) < num_tiles) {
-      int m0, n0, expert, row_end;
-      coords(blockIdx.x, m0, n0, expert, row_end);
-      pre = KB < C::kStages ? KB : C::kStages;
-      if (lane == 0) {
+    if (lane == 0) {
+      int pre = 0;
+      bool half0 = true;
+      int m0p = 0, n0p = 0, ep = 0, rep_end = 0;
+      if (static_cast<int>(blockIdx.x) < num_tiles) coords(blockIdx.x, m0p, n0p, ep, rep_end, half0);
+      if (!kGrouped && early_b && static_cast<int>(blockIdx.x) < num_tiles && !half0) {
+        const int n0 = n0p;
+        pre = KB < C::kStages ? KB : C::kStages;
         for (int kb = 0; kb < pre; ++kb) {
           mbar_arrive_expect_tx(&full[kb], C::kStageBytes);
           tma_load_2d(sB + kb * C::kBBytes, &tmB, &full[kb], kb * C::kBK, n0);
         }
       }
-    }
-    griddep_wait();
-    uint32_t it = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-      int m0, n0, expert, row_end;
-      coords(t, m0, n0, expert, row_end);
-      if (expert < 0) {
-        if (lane == 0 && expert == -1) record_status(kDevBadGroupOffsets);
-        continue;
-      }
-      const uint64_t ws_row = (static_cast<uint64_t>(expert) * NB + n0 / 128) * KB;
-      // prefetched scale bytes: rows lane + 32 j of the tile's A rows, and the
-      // scale of each 128-row weight block of the tile
-      uint32_t pa[C::kPrefetch][4], pw[C::kPrefetch][BN / 128];
-      auto fetch = [&](int kb, uint32_t (&a)[4], uint32_t (&w)[BN / 128]) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int m = m0 + lane + 32 * j;
-          a[j] = (kb < KB && m < row_end) ? __ldg(Xs + static_cast<uint64_t>(kb) * ld_s + m) : 127u;
+      griddep_wait();
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        int m0, n0, expert, row_end;
+        bool half;
+        coords(t, m0, n0, expert, row_end, half);
+        if (expert < 0) {
+          if (expert == -1) record_status(kDevBadGroupOffsets);
+          continue;
         }
-#pragma unroll
-        for (int h = 0; h < BN / 128; ++h) w[h] = kb < KB ? __ldg(Ws + ws_row + static_cast<uint64_t>(h) * KB + kb) : 127u;
-      };
-#pragma unroll
-      for (int d = 0; d < C::kPrefetch; ++d) fetch(d, pa[d], pw[d]);
-      for (int kb0 = 0; kb0 < KB && ok; kb0 += C::kPrefetch) {
-#pragma unroll
-        for (int d = 0; d < C::kPrefetch; ++d) {
-          const int kb = kb0 + d;
-          if (kb >= KB) break;
+        const CUtensorMap* mapB = (kHalfTiles && half) ? &tmBh : &tmB;
+        const uint32_t stage_tx = (kHalfTiles && half) ? C::kABytes + C::kBBytes / 2 : C::kStageBytes;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % C::kStages;
-          if (!__all_sync(0xFFFFFFFFu, it < static_cast<uint32_t>(C::kStages) ||
-                                           mbar_wait(&empty[s], ((it / C::kStages) & 1u) ^ 1u))) {
-            if (lane == 0) record_status(kDevTimeoutProducer);
+          if (it >= static_cast<uint32_t>(C::kStages) && !mbar_wait(&empty[s], ((it / C::kStages) & 1u) ^ 1u)) {
+            record_status(kDevTimeoutProducer);
             ok = false;
             break;
           }
-          if (lane == 0) {
-            if (it >= static_cast<uint32_t>(pre)) {
-              mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-              tma_load_2d(sB + s * C::kBBytes, &tmB, &full[s], kb * C::kBK, expert * N + n0);
-            }
-            tma_load_2d(sA + s * C::kABytes, &tmA, &full[s], kb * C::kBK, m0);
+          if (it >= static_cast<uint32_t>(pre)) {
+            mbar_arrive_expect_tx(&full[s], stage_tx);
+            tma_load_2d(sB + s * C::kBBytes, mapB, &full[s], kb * C::kBK, expert * N + n0);
           }
-          // scale rows in the TMEM scale layout: lane l holds rows l + 32 j,
-          // each byte repeated for the four 32-element K slices
-          uint4 ra;
-          ra.x = pa[d][0] * 0x01010101u;
-          ra.y = pa[d][1] * 0x01010101u;
-          ra.z = pa[d][2] * 0x01010101u;
-          ra.w = pa[d][3] * 0x01010101u;
-          *reinterpret_cast<uint4*>(sSfA + s * C::kSfABytes + lane * 16) = ra;
-#pragma unroll
-          for (int h = 0; h < BN / 128; ++h) {
-            const uint32_t w4 = pw[d][h] * 0x01010101u;
-            *reinterpret_cast<uint4*>(sSfB + s * C::kSfBBytes + h * 512 + lane * 16) = make_uint4(w4, w4, w4, w4);
-          }
-          fetch(kb + C::kPrefetch, pa[d], pw[d]);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&full[s]);
-          ++it;
+          tma_load_2d(sA + s * C::kABytes, &tmA, &full[s], kb * C::kBK, m0);
         }
       }
-    }
-    if (lane == 0) {
       for (uint32_t j = (it > static_cast<uint32_t>(C::kStages) ? it - C::kStages : 0); j < it; ++j)
         if (!mbar_wait(&full[j % C::kStages], (j / C::kStages) & 1u)) record_status(kDevTimeoutProducer);
+    }
+  } else if (warp == 2) {
+    // ================= scale groups into shared memory (all lanes)
+    uint32_t grp = 0;                          // scale groups issued so far
+    bool ok = true;
+    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      int m0, n0, expert, row_end;
+      bool half;
+      coords(t, m0, n0, expert, row_end, half);
+      if (expert < 0) continue;
+      const int nblk = (kHalfTiles && half) ? 1 : BN / 128;   // weight blocks the tile covers
+      const uint64_t ws_row = (static_cast<uint64_t>(expert) * NB + n0 / 128) * KB;
+      // Scale group g = K blocks 4g .. 4g+3, byte b of every word for K block
+      // 4g + b: rows lane + 32 j of the tile's A rows (ra[.][j][b]) and the
+      // scale of the tile's 128-row weight block h (rw[.][h][b]).  Groups go
+      // out kSfBatch at a time (one proxy fence per batch); the raw bytes
+      // are fetched one batch ahead and packed only when written.
+      uint32_t ra[C::kSfBatch][4][C::kSfGroup], rw[C::kSfBatch][BN / 128][C::kSfGroup];
+      auto fetch = [&](int g0) {
+#pragma unroll
+        for (int q = 0; q < C::kSfBatch; ++q) {
+#pragma unroll
+          for (int b = 0; b < C::kSfGroup; ++b) {
+            const int kb = (g0 + q) * C::kSfGroup + b;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int m = m0 + lane + 32 * j;
+              ra[q][j][b] = (kb < KB && m < row_end) ? __ldg(Xs + static_cast<uint64_t>(kb) * ld_s + m) : 127u;
+            }
+#pragma unroll
+            for (int h = 0; h < BN / 128; ++h)
+              rw[q][h][b] = (kb < KB && h < nblk) ? __ldg(Ws + ws_row + static_cast<uint64_t>(h) * KB + kb) : 127u;
+          }
+        }
+      };
+      auto pack = [](const uint32_t (&v)[C::kSfGroup]) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int b = 0; b < C::kSfGroup; ++b) word |= v[b] << (8 * b);
+        return word;
+      };
+      const int groups = (KB + C::kSfGroup - 1) / C::kSfGroup;
+      fetch(0);
+      for (int g0 = 0; g0 < groups; g0 += C::kSfBatch) {
+        const int nb = groups - g0 < C::kSfBatch ? groups - g0 : C::kSfBatch;
+        // slot (grp + q) % kSfSlots is free once the copy of group
+        // grp + q - kSfSlots is done
+        bool free = true;
+        for (int q = 0; q < nb; ++q) {
+          const uint32_t gq = grp + q;
+          free = free && (gq < static_cast<uint32_t>(C::kSfSlots) ||
+                          mbar_wait(&sf_empty[gq % C::kSfSlots], ((gq / C::kSfSlots) & 1u) ^ 1u));
+        }
+        if (!__all_sync(0xFFFFFFFFu, free)) {
+          if (lane == 0) record_status(kDevTimeoutProducer);
+          ok = false;
+          break;
+        }
+        // the TMEM scale layout: lane l holds rows l + 32 j (word j), a
+        // weight tile its block's word in every position
+#pragma unroll
+        for (int q = 0; q < C::kSfBatch; ++q) {
+          if (q < nb) {
+            const int sl = static_cast<int>((grp + q) % C::kSfSlots);
+            *reinterpret_cast<uint4*>(sSfA + sl * C::kSfABytes + lane * 16) =
+                make_uint4(pack(ra[q][0]), pack(ra[q][1]), pack(ra[q][2]), pack(ra[q][3]));
+#pragma unroll
+            for (int h = 0; h < BN / 128; ++h) {
+              const uint32_t w = pack(rw[q][h]);
+              *reinterpret_cast<uint4*>(sSfB + sl * C::kSfBBytes + h * 512 + lane * 16) = make_uint4(w, w, w, w);
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0)
+          for (int q = 0; q < nb; ++q) mbar_arrive(&sf_full[(grp + q) % C::kSfSlots]);
+        grp += nb;
+        fetch(g0 + C::kSfBatch);
+      }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ================= MMA issuer
-      constexpr uint32_t idesc = idesc_mx_e4m3_ue8m0(128, C::kBN);
+      // K block kb reads byte kb % 4 of its group's scale words (scale
+      // factor ids in the instruction descriptor: A bits 29-30, B bits 4-5)
+      constexpr uint32_t idesc0 = idesc_mx_e4m3_ue8m0(128, C::kBN);
+      constexpr uint32_t idesc_half = idesc_mx_e4m3_ue8m0(128, C::kBN / 2);
       const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
       // descriptors differ per stage / K step only in the start-address field
       const uint64_t a_desc0 = smem_desc_k_sw128(a_base), b_desc0 = smem_desc_k_sw128(b_base);
       const uint64_t sfa_desc0 = smem_desc_rows16(smem_u32(sSfA)), sfb_desc0 = smem_desc_rows16(smem_u32(sSfB));
-      uint32_t it = 0, tile_no = 0;
+      uint32_t it = 0, grp = 0, tile_no = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         int m0, n0, expert, row_end;
-        coords(t, m0, n0, expert, row_end);
+        bool half;
+        coords(t, m0, n0, expert, row_end, half);
         if (expert < 0) continue;
+        const uint32_t idesc_t = (kHalfTiles && half) ? idesc_half : idesc0;
         const int ab = tile_no % C::kNumAcc;            // accumulator buffer
         const int tb = tile_no & 1;                      // tfull / tempty barrier of this tile
         if (tile_no >= static_cast<uint32_t>(C::kNumAcc) &&
@@ -904,27 +980,43 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d = tmem_base + static_cast<uint32_t>(ab * C::kBN);
-        for (int kb = 0; kb < KB; ++kb, ++it) {
-          const int s = it % C::kStages;
-          if (!mbar_wait(&full[s], (it / C::kStages) & 1u)) {
+        // per scale group: its copy into TMEM slot grp % kSfSlots (in issue
+        // order with the MMAs, which read the previous group's slot), then the
+        // group's K blocks; K block kb reads byte kb % 4 of the scale words
+        for (int kb0 = 0; kb0 < KB && ok; kb0 += C::kSfGroup, ++grp) {
+          const int sl = static_cast<int>(grp % C::kSfSlots);
+          if (!mbar_wait(&sf_full[sl], (grp / C::kSfSlots) & 1u)) {
             record_status(kDevTimeoutMma);
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sfa = tmem_base + C::kSfCol + static_cast<uint32_t>((kb & 1) * C::kSfColsPerKb);
+          const uint32_t sfa = tmem_base + C::kSfCol + static_cast<uint32_t>(sl * C::kSfColsPerSlot);
           const uint32_t sfb = sfa + 4;
-          tmem_cp_32x128b_x4(sfa, sfa_desc0 + ((s * C::kSfABytes) >> 4));
+          tmem_cp_32x128b_x4(sfa, sfa_desc0 + ((sl * C::kSfABytes) >> 4));
 #pragma unroll
           for (int h = 0; h < BN / 128; ++h)
-            tmem_cp_32x128b_x4(sfb + 4 * h, sfb_desc0 + ((s * C::kSfBBytes + h * 512) >> 4));
+            tmem_cp_32x128b_x4(sfb + 4 * h, sfb_desc0 + ((sl * C::kSfBBytes + h * 512) >> 4));
+          mma_commit(&sf_empty[sl]);                     // the slot may be refilled once copied
+          const int kb1 = kb0 + C::kSfGroup < KB ? kb0 + C::kSfGroup : KB;
+          for (int kb = kb0; kb < kb1; ++kb, ++it) {
+            const int s = it % C::kStages;
+            if (!mbar_wait(&full[s], (it / C::kStages) & 1u)) {
+              record_status(kDevTimeoutMma);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sf_id = static_cast<uint32_t>(kb - kb0);
+            const uint32_t idesc = idesc_t | (sf_id << 29) | (sf_id << 4);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t adesc = a_desc0 + ((s * C::kABytes + kk * 32) >> 4);
-            const uint64_t bdesc = b_desc0 + ((s * C::kBBytes + kk * 32) >> 4);
-            mma_mxf8f6f4(d, adesc, bdesc, idesc, sfa, sfb, (kb > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t adesc = a_desc0 + ((s * C::kABytes + kk * 32) >> 4);
+              const uint64_t bdesc = b_desc0 + ((s * C::kBBytes + kk * 32) >> 4);
+              mma_mxf8f6f4(d, adesc, bdesc, idesc, sfa, sfb, (kb > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(&empty[s]);
           }
-          mma_commit(&empty[s]);
         }
         if (ok) mma_commit(&tfull[tb]);
         ++tile_no;
@@ -941,7 +1033,8 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
     uint32_t tile_no = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
       int m0, n0, expert, row_end;
-      coords(t, m0, n0, expert, row_end);
+      bool half;
+      coords(t, m0, n0, expert, row_end, half);
       if (expert < 0) continue;
       const int ab = tile_no % C::kNumAcc;
       const int tb = tile_no & 1;
@@ -950,6 +1043,14 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
         break;
       }
       tc_fence_after();
+      if (kHalfTiles && half && col0 >= C::kBN / 2) {
+        // no columns of this half tile: hand the accumulator back at once
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[tb]);
+        ++tile_no;
+        continue;
+      }
       const int m = m0 + row;
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(ab * C::kBN + col0);

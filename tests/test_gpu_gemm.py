@@ -83,17 +83,19 @@ def test_gemm_zero_and_unit_codes(dev):
     assert (Y.float() == 0).all()
 
 
-@pytest.mark.parametrize("M,N,K", [(1200, 4096, 256), (2560, 2304, 384)])
-def test_gemm_half_tile_tail(dev, M, N, K):
+@pytest.mark.parametrize("fmt", [F32, UE8M0])
+@pytest.mark.parametrize("M,N,K", [(1200, 4096, 256), (2560, 2304, 384), (1200, 4096, 1152)])
+def test_gemm_half_tile_tail(dev, M, N, K, fmt):
     """Shapes whose last partial wave of 128x256 tiles runs as 128x128 half
     tiles on a 148-SM B200 (1200x4096: 160 tiles = 148 + 12, ragged last
-    M tile; 2560x2304: 180 tiles = 148 + 32): every output against the
-    oracle."""
+    M tile; 2560x2304: 180 tiles = 148 + 32), in both scale formats (the
+    UE8M0 kernel's scale groups of four K blocks: K = 1152 ends in a group
+    of one): every output against the oracle."""
     cfg = workloads.scaled_linear(workloads.TINY, M=M, N=N, K=K, seed=M + N + K)
     X, W = workloads.linear_inputs(cfg)
-    Y = gpu_linear(X.to(dev), W.to(dev), F32)
-    Y_ref, S = oracle_linear(bits16(X), bits16(W), F32)
-    assert_gemm_close(y_to_f64(Y), Y_ref, S, f"half-tile tail {M}x{N}x{K}")
+    Y = gpu_linear(X.to(dev), W.to(dev), fmt)
+    Y_ref, S = oracle_linear(bits16(X), bits16(W), fmt)
+    assert_gemm_close(y_to_f64(Y), Y_ref, S, f"half-tile tail {M}x{N}x{K} fmt {fmt}")
 
 
 def sample_rows(M, n_random=48, seed=0):
@@ -103,8 +105,8 @@ def sample_rows(M, n_random=48, seed=0):
     return np.unique(rows)
 
 
-@pytest.mark.parametrize("cfg", [workloads.LLAMA_ATTN, workloads.LLAMA_GATE_UP, workloads.LLAMA_DOWN],
-                         ids=lambda c: c.name)
+@pytest.mark.parametrize("cfg", [workloads.LLAMA_ATTN, workloads.LLAMA_GATE_UP, workloads.LLAMA_DOWN,
+                                 *workloads.LLAMA_UE8M0.values()], ids=lambda c: c.name)
 def test_gemm_full_size_sampled_rows(dev, cfg):
     X = workloads.activations((cfg.M, cfg.K), cfg.x_kind, cfg.seed, device=dev)
     W = workloads.weights((cfg.N, cfg.K), cfg.seed + 1, device=dev)

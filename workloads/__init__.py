@@ -20,7 +20,7 @@ a test always feeds the oracle the same bytes the GPU saw.
 """
 from __future__ import annotations
 
-from dataclasses import dataclass, field
+from dataclasses import dataclass, field, replace
 
 import numpy as np
 import torch
@@ -71,7 +71,12 @@ MOE_SMALL = MoE("deepseek_v3_moe_32x4096x7168_top8_512tok", E=32, tokens=512)
 MOE_DECODE = MoE("deepseek_v3_moe_decode_masked_256x4096x7168_top8_128tok", tokens=128)
 MOE_DECODE_SMALL = MoE("deepseek_v3_moe_decode_masked_32x4096x7168_top8_64tok", E=32, tokens=64)
 
-LINEARS = {c.name: c for c in [TINY, LLAMA_ATTN, LLAMA_GATE_UP, LLAMA_DOWN, *DS_DECODE.values()]}
+# the dense prefill shapes with power-of-two (UE8M0) scales: the tensor core's
+# block-scaled MMA path instead of the fp32 promotion
+LLAMA_UE8M0 = {c.name: replace(c, name=f"{c.name}_ue8m0", fmt=SCALE_UE8M0)
+               for c in (LLAMA_ATTN, LLAMA_GATE_UP, LLAMA_DOWN)}
+LINEARS = {c.name: c for c in [TINY, LLAMA_ATTN, LLAMA_GATE_UP, LLAMA_DOWN, *DS_DECODE.values(),
+                               *LLAMA_UE8M0.values()]}
 
 
 def _gen(device, seed: int) -> torch.Generator:
