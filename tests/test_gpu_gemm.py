@@ -169,6 +169,22 @@ def test_grouped_gemm_small(dev, fmt):
     assert (Y[pad].float() == 0).all()
 
 
+@pytest.mark.parametrize("fmt", [UE8M0, F32])
+def test_grouped_gemm_every_row_mixed_experts(dev, fmt):
+    """Zipf-routed experts with many row tiles and experts with one (the
+    UE8M0 kernel interleaves the two kinds of row tiles in its schedule):
+    every token row against the oracle, every padding row zero."""
+    cfg = workloads.scaled_moe(workloads.MOE, E=48, N=256, K=512, tokens=1024, topk=6, fmt=fmt)
+    r, X, Y = build_moe(cfg, dev)
+    tiles = np.diff(r.group_offs) // 128
+    assert (tiles >= 2).any() and (tiles == 1).any()
+    valid = np.where(r.row_token >= 0)[0]
+    Y_ref, S = oracle_moe_rows(cfg, r, X, valid, dev)
+    assert_gemm_close(y_to_f64(Y[torch.as_tensor(valid, device=dev)]), Y_ref, S, "grouped mixed experts")
+    pad = torch.as_tensor(np.where(r.row_token < 0)[0], device=dev)
+    assert (Y[pad].float() == 0).all()
+
+
 def test_grouped_gemm_empty_experts(dev):
     """Experts with no rows (zero-length segments) are skipped."""
     cfg = workloads.scaled_moe(workloads.MOE, E=40, N=128, K=256, tokens=20, topk=1, zipf=3.0)
