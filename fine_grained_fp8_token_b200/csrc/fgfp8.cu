@@ -293,12 +293,39 @@ fgfp8_status launch_decode(const uint8_t* Xq, const void* Xs, int64_t ld_s, cons
                           static_cast<int>(K), early);
 }
 
+// UE8M0 few-token launch: the block-scaled MMA applies the scales.
+template <int BNT>
+fgfp8_status launch_decode_mx(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
+                              void* Y, int64_t M, int64_t N, int64_t K, cudaStream_t stream, int dev, int early) {
+  using C = fgfp8::DecodeMxCfg<BNT>;
+  CUtensorMap mX, mW;
+  fgfp8_status st = make_map_u8_sw128(&mX, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
+                                      static_cast<uint64_t>(K), BNT);
+  if (st != FGFP8_OK) return st;
+  st = make_map_u8_sw128(&mW, Wq, static_cast<uint64_t>(N), static_cast<uint64_t>(K), static_cast<uint64_t>(K), 128);
+  if (st != FGFP8_OK) return st;
+  auto kernel = fgfp8::gemm_decode_mx_kernel<BNT>;
+  st = set_smem(reinterpret_cast<const void*>(kernel), C::kSmemBytes, dev);
+  if (st != FGFP8_OK) return st;
+  return launch_dependent(kernel, static_cast<unsigned>(N / 128), C::kThreads, C::kSmemBytes, stream,
+                          "decode gemm launch", mX, mW, reinterpret_cast<const uint8_t*>(Xs),
+                          static_cast<uint32_t>(ld_s), reinterpret_cast<const uint8_t*>(Ws),
+                          reinterpret_cast<__nv_bfloat16*>(Y), static_cast<int>(M), static_cast<int>(N),
+                          static_cast<int>(K), early);
+}
+
 template <int FMT>
 fgfp8_status dispatch_decode(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
                              void* Y, int64_t M, int64_t N, int64_t K, cudaStream_t s, int dev, int early) {
-  if (M <= 16) return launch_decode<16, FMT>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev, early);
-  if (M <= 32) return launch_decode<32, FMT>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev, early);
-  return launch_decode<64, FMT>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev, early);
+  if constexpr (FMT == FGFP8_SCALE_UE8M0) {
+    if (M <= 16) return launch_decode_mx<16>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev, early);
+    if (M <= 32) return launch_decode_mx<32>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev, early);
+    return launch_decode_mx<64>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev, early);
+  } else {
+    if (M <= 16) return launch_decode<16, FMT>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev, early);
+    if (M <= 32) return launch_decode<32, FMT>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev, early);
+    return launch_decode<64, FMT>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, s, dev, early);
+  }
 }
 
 // Row/column-scaled GEMM: persistent grid of 128 x BN tiles.

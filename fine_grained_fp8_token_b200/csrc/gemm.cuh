@@ -1481,4 +1481,229 @@ __global__ void __launch_bounds__(DecodeCfg<BNT>::kThreads, 1)
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
 }
 
+// ---------------------------------------------------------------------------
+// Few-token GEMM with UE8M0 scales on the block-scaled MMA ("UE8M0 scale
+// format": power-of-two scales the tensor core applies itself).  Operands
+// swapped as in gemm_decode_kernel: the CTA's 128 weight rows are the MMA's
+// M, the BNT token rows its N.  Every A row takes the weight block's scale,
+// every B row its token's 1x128 group scale, so the whole K reduction
+// accumulates in TMEM and nothing but the scale words runs per K block off
+// the tensor pipe (groups of four K blocks, byte b of each word for K block
+// 4g + b, as in gemm_mx_kernel).
+//   warp 0      TMA: per K block the 128-row weight tile and the token tile
+//               (rows >= M read as zeros);
+//   warp 1      TMEM owner and MMA issuer: per scale group tcgen05.cp of
+//               the two scale tiles, per K block four block-scaled MMAs;
+//   warp 2      the scale words into shared memory, two groups per fence;
+//   warps 4..7  epilogue: the BNT finished columns of their 32 weight rows,
+//               stored transposed into Y[m, n].
+// ---------------------------------------------------------------------------
+template <int BNT>
+struct DecodeMxCfg {
+  static constexpr uint32_t kABytes = 128 * 128;             // weight tile
+  static constexpr uint32_t kBBytes = BNT * 128;             // token tile
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = (192 * 1024) / kStageBytes > 12 ? 12 : (192 * 1024) / kStageBytes;
+  static constexpr int kSfGroup = 4;                         // K blocks per scale word
+  static constexpr int kSfBatch = 2;                         // groups per shared-memory fence
+  static constexpr int kSfSlots = 2 * kSfBatch;
+  static constexpr uint32_t kSfTileBytes = 512;              // one 32 x 16-byte scale tile
+  static constexpr int kThreads = 8 * 32;
+  static constexpr uint32_t kSfCol = BNT < 32 ? 32 : BNT;    // scale slots after the accumulator
+  static constexpr uint32_t kSfColsPerSlot = 8;              // A: 4 columns, B: 4 columns
+  static constexpr uint32_t kTmemCols = (kSfCol + kSfSlots * kSfColsPerSlot) <= 64 ? 64 : 128;
+  static constexpr size_t kBarrierBytes = 256;
+  static constexpr size_t kSmemBytes =
+      1024 + kStages * static_cast<size_t>(kStageBytes) + kSfSlots * 2 * static_cast<size_t>(kSfTileBytes) + kBarrierBytes;
+};
+
+template <int BNT>
+__global__ void __launch_bounds__(DecodeMxCfg<BNT>::kThreads, 1)
+    gemm_decode_mx_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                          const uint8_t* __restrict__ Xs, uint32_t ld_s, const uint8_t* __restrict__ Ws,
+                          __nv_bfloat16* __restrict__ Y, int M, int N, int K, int early_w) {
+  using C = DecodeMxCfg<BNT>;
+  static_assert(C::kSfCol + C::kSfSlots * C::kSfColsPerSlot <= C::kTmemCols, "TMEM columns");
+  static_assert((2 * C::kStages + 1 + 1 + 2 * C::kSfSlots) * 8 + 4 <= C::kBarrierBytes, "barrier area");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sW = smem;
+  uint8_t* sX = smem + C::kStages * C::kABytes;
+  uint8_t* sSfA = sX + C::kStages * C::kBBytes;                 // weight-block scale tiles, per slot
+  uint8_t* sSfB = sSfA + C::kSfSlots * C::kSfTileBytes;         // token scale tiles, per slot
+  uint64_t* full = reinterpret_cast<uint64_t*>(sSfB + C::kSfSlots * C::kSfTileBytes);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
+  uint64_t* mma_done = tfull + 1;
+  uint64_t* sf_full = mma_done + 1;
+  uint64_t* sf_empty = sf_full + C::kSfSlots;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_empty + C::kSfSlots);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int KB = K / 128;
+  const int n0 = blockIdx.x * 128;
+  const int groups = (KB + C::kSfGroup - 1) / C::kSfGroup;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(tfull, 1);
+    mbar_init(mma_done, 1);
+    for (int b = 0; b < C::kSfSlots; ++b) {
+      mbar_init(&sf_full[b], 1);
+      mbar_init(&sf_empty[b], 1);
+    }
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  // Dependency on the preceding grid (programmatic launch): the producer may
+  // request the first weight tiles before it; every other access follows it.
+  if (threadIdx.x != 0) griddep_wait();
+  if (warp == 0) {
+    if (lane == 0)
+      produce_tiles<C::kStages, C::kABytes, C::kBBytes>(&tmW, n0, &tmX, 0, KB, sW, sX, full, empty, early_w != 0);
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ================= MMA issuer
+      constexpr uint32_t idesc0 = idesc_mx_e4m3_ue8m0(128, BNT);
+      const uint64_t a_desc0 = smem_desc_k_sw128(smem_u32(sW)), b_desc0 = smem_desc_k_sw128(smem_u32(sX));
+      const uint64_t sfa_desc0 = smem_desc_rows16(smem_u32(sSfA)), sfb_desc0 = smem_desc_rows16(smem_u32(sSfB));
+      bool ok = true;
+      uint32_t it = 0;
+      for (int g = 0; g < groups && ok; ++g) {
+        const int sl = g % C::kSfSlots;
+        if (!mbar_wait(&sf_full[sl], (g / C::kSfSlots) & 1u)) {
+          record_status(kDevTimeoutMma);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sfa = tmem_base + C::kSfCol + static_cast<uint32_t>(sl * C::kSfColsPerSlot);
+        const uint32_t sfb = sfa + 4;
+        tmem_cp_32x128b_x4(sfa, sfa_desc0 + ((sl * C::kSfTileBytes) >> 4));
+        tmem_cp_32x128b_x4(sfb, sfb_desc0 + ((sl * C::kSfTileBytes) >> 4));
+        mma_commit(&sf_empty[sl]);                     // the slot may be refilled once copied
+        const int kb0 = g * C::kSfGroup, kb1 = kb0 + C::kSfGroup < KB ? kb0 + C::kSfGroup : KB;
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % C::kStages;
+          if (!mbar_wait(&full[s], (it / C::kStages) & 1u)) {
+            record_status(kDevTimeoutMma);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sf_id = static_cast<uint32_t>(kb - kb0);
+          const uint32_t idesc = idesc0 | (sf_id << 29) | (sf_id << 4);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t adesc = a_desc0 + ((s * C::kABytes + kk * 32) >> 4);
+            const uint64_t bdesc = b_desc0 + ((s * C::kBBytes + kk * 32) >> 4);
+            mma_mxf8f6f4(tmem_base, adesc, bdesc, idesc, sfa, sfb, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&empty[s]);
+        }
+      }
+      if (ok) mma_commit(tfull);
+      mma_commit(mma_done);
+      if (!mbar_wait(mma_done, 0)) record_status(kDevTimeoutMma);
+    }
+  } else if (warp == 2) {
+    // ================= scale words into shared memory (all lanes)
+    // Group g: the weight block's word (byte b: K block 4g + b) in every
+    // position of the A tile; B tile lane l, word j: token l + 32 j (127 =
+    // 2^0 past M; rows >= BNT are never read).  Raw bytes one batch ahead.
+    const uint64_t ws_row = static_cast<uint64_t>(n0 / 128) * KB;
+    uint32_t ra[C::kSfBatch][4][C::kSfGroup], rw[C::kSfBatch][C::kSfGroup];
+    auto fetch = [&](int g0) {
+#pragma unroll
+      for (int q = 0; q < C::kSfBatch; ++q) {
+#pragma unroll
+        for (int b = 0; b < C::kSfGroup; ++b) {
+          const int kb = (g0 + q) * C::kSfGroup + b;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int m = lane + 32 * j;
+            ra[q][j][b] = (kb < KB && m < M && m < BNT) ? __ldg(Xs + static_cast<uint64_t>(kb) * ld_s + m) : 127u;
+          }
+          rw[q][b] = kb < KB ? __ldg(Ws + ws_row + kb) : 127u;
+        }
+      }
+    };
+    auto pack = [](const uint32_t (&v)[C::kSfGroup]) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int b = 0; b < C::kSfGroup; ++b) word |= v[b] << (8 * b);
+      return word;
+    };
+    fetch(0);
+    for (int g0 = 0; g0 < groups; g0 += C::kSfBatch) {
+      const int nb = groups - g0 < C::kSfBatch ? groups - g0 : C::kSfBatch;
+      bool free = true;
+      for (int q = 0; q < nb; ++q) {
+        const int gq = g0 + q;
+        free = free && (gq < C::kSfSlots || mbar_wait(&sf_empty[gq % C::kSfSlots], ((gq / C::kSfSlots) & 1) ^ 1));
+      }
+      if (!__all_sync(0xFFFFFFFFu, free)) {
+        if (lane == 0) record_status(kDevTimeoutProducer);
+        break;
+      }
+#pragma unroll
+      for (int q = 0; q < C::kSfBatch; ++q) {
+        if (q < nb) {
+          const int sl = (g0 + q) % C::kSfSlots;
+          const uint32_t w = pack(rw[q]);
+          *reinterpret_cast<uint4*>(sSfA + sl * C::kSfTileBytes + lane * 16) = make_uint4(w, w, w, w);
+          *reinterpret_cast<uint4*>(sSfB + sl * C::kSfTileBytes + lane * 16) =
+              make_uint4(pack(ra[q][0]), pack(ra[q][1]), pack(ra[q][2]), pack(ra[q][3]));
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0)
+        for (int q = 0; q < nb; ++q) mbar_arrive(&sf_full[(g0 + q) % C::kSfSlots]);
+      fetch(g0 + C::kSfBatch);
+    }
+  } else if (warp >= 4) {
+    // ================= epilogue
+    const int quad = warp & 3;
+    const int n = n0 + quad * 32 + lane;
+    if (__all_sync(0xFFFFFFFFu, mbar_wait(tfull, 0))) {
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+      uint32_t p[BNT];
+#pragma unroll
+      for (int c = 0; c < BNT / 16; ++c)
+        tmem_ld_32x32b_x16(taddr + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&p[c * 16]));
+      tmem_wait_ld();
+      if (n < N) {
+#pragma unroll
+        for (int m = 0; m < BNT; ++m)
+          if (m < M) Y[static_cast<uint64_t>(m) * N + n] = __float2bfloat16_rn(__uint_as_float(p[m]));
+      }
+    } else if (lane == 0) {
+      record_status(kDevTimeoutEpilogue);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
 }  // namespace fgfp8
