@@ -249,7 +249,7 @@ class DenseLayer:
 
     def gemm_kernel_name(self):
         if self.cfg.M <= 64:
-            return "gemm_decode_kernel"
+            return "gemm_decode_kernel" if self.cfg.fmt == 0 else "gemm_decode_mx_kernel"
         return "gemm_blockscaled_kernel" if self.cfg.fmt == 0 else "gemm_mx_kernel"
 
 
