@@ -1332,8 +1332,9 @@ __global__ void __launch_bounds__(RowColCfg<BN>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Few-token variant (M <= 64, decode): operands swapped so the weight supplies
-// the MMA's 128 rows and the tokens its N dimension (BNT = M rounded up to
+// Few-token variant with fp32 scales (M <= 64, decode; UE8M0 scales take
+// gemm_decode_mx_kernel below): operands swapped so the weight supplies the
+// MMA's 128 rows and the tokens its N dimension (BNT = M rounded up to
 // 16/32/64).  One CTA streams one 128-row weight slab through a deep TMA ring
 // (the layer is bound by reading Wq from HBM).  TMEM holds D^T: lane = output
 // column n, column = token m.  Each promotion thread owns one n and BNT
