@@ -90,3 +90,36 @@ def test_masked_bad_count_reported(dev):
     assert (Y[cap:2 * cap].float() == SENTINEL).all()          # the bad expert's rows untouched
     check_rows(X, W_list, Y, [5, 0, 128], cap, F32, "bad-count neighbours")
     fg.check_device_status()                                    # cleared
+
+
+def test_masked_full_decode_step_sampled_experts(dev):
+    """The 256-expert decode step the benchmark times (128 tokens top-8,
+    Zipf-routed, cap = 128, UE8M0): every token row of the busiest experts,
+    a middle one and the last active one against the oracle, every padding
+    row of every expert untouched."""
+    cfg, cap = workloads.MOE_DECODE, 128
+    r = workloads.moe_routing(cfg)
+    X = workloads.moe_masked_rows(workloads.moe_tokens(cfg, device=dev), r, cfg.E, cap)
+    Wq = torch.empty((cfg.E, cfg.N, cfg.K), dtype=torch.uint8, device=dev)
+    Ws = torch.empty((cfg.E, cfg.N // 128, cfg.K // 128), dtype=torch.uint8, device=dev)
+    for e in range(cfg.E):
+        fg.quant_weight(workloads.moe_expert_weight(cfg, e, device=dev), UE8M0, Wq=Wq[e], Ws=Ws[e])
+    Xq, Xs = fg.quant_act(X, UE8M0)
+    cnt = torch.as_tensor(r.counts.astype(np.int32), device=dev)
+    Y = torch.full((cfg.E * cap, cfg.N), SENTINEL, dtype=torch.bfloat16, device=dev)
+    fg.masked_gemm(Xq, Xs, Wq, Ws, cnt, UE8M0, Y=Y)
+    fg.check_device_status()
+    active = np.where(r.counts > 0)[0]
+    pick = np.unique(np.r_[np.argsort(-r.counts)[:3], active[len(active) // 2], active[-1]])
+    for e in pick:
+        c = int(r.counts[e])
+        rows = slice(int(e) * cap, int(e) * cap + c)
+        Xq_r, Xs_r = oracle.quant_act(bits16(X[rows]), UE8M0)
+        Wq_r, Ws_r = oracle.quant_weight(bits16(workloads.moe_expert_weight(cfg, int(e), device=dev)), UE8M0)
+        Y_ref, S = oracle.gemm(Xq_r, Xs_r, Wq_r, Ws_r, UE8M0)
+        assert_gemm_close(y_to_f64(Y[rows]), Y_ref, S, f"masked decode expert {e}")
+    pad = torch.ones(cfg.E * cap, dtype=torch.bool, device=dev)
+    for e in active:
+        pad[int(e) * cap:int(e) * cap + int(r.counts[e])] = False
+    assert (Y[pad].float() == SENTINEL).all(), "padding rows written"
+

@@ -87,6 +87,30 @@ def test_swiglu_quant_against_oracle(dev, M, I, K):
     check_against_oracle(to_np(Hq), to_np(Hs), g, u, Sg, Su, M, I)
 
 
+def test_swiglu_quant_full_mlp_sampled_rows(dev):
+    """The Llama-3-8B MLP's gate/up projection at full size (8192 tokens,
+    K = 4096, I = 14336, the inputs the MLP benchmark builds): every M tile's
+    first and last row plus random rows against the oracle, with the same
+    bounds as above."""
+    c = workloads.LLAMA_GATE_UP
+    M, K, I = 8192, 4096, 14336
+    X = workloads.activations((M, K), c.x_kind, c.seed, device=dev)
+    Wg = workloads.weights((I, K), c.seed + 1, device=dev)
+    Wu = workloads.weights((I, K), c.seed + 2, device=dev)
+    W_gu = fg.interleave_gate_up(Wg, Wu)
+    del Wg, Wu
+    Xq, Xs = fg.quant_act(X, F32)
+    Wq, Ws = fg.quant_weight(W_gu, F32)
+    Hq, Hs = fg.gemm_swiglu_quant(Xq, Xs, Wq, Ws)
+    fg.check_device_status()
+    rng = np.random.default_rng(1)
+    tiles = np.arange(0, M, 128)
+    rows = np.unique(np.concatenate([tiles[::4], tiles[::4] + 127, rng.integers(0, M, 8)]))
+    idx = torch.as_tensor(rows, device=dev)
+    g, u, Sg, Su = oracle_h(X[idx], W_gu, I)
+    check_against_oracle(to_np(Hq[idx]), to_np(Hs[:, idx]), g, u, Sg, Su, len(rows), I)
+
+
 def host_swiglu_quant(Y_gu: torch.Tensor, I: int):
     """The unfused path's last two steps on the host: SiLU(g) * u in fp32 from
     the bf16 GEMM output, rounded to bf16, then the 1x128 quantizer."""
