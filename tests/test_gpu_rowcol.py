@@ -127,6 +127,30 @@ def test_gemm_rowcol_full_size_sampled_rows(dev, cfg):
     assert_gemm_close(y_to_f64(Y[torch.as_tensor(rows, device=dev)]), Y_ref, S, f"FP8_DYNAMIC {cfg.name}")
 
 
+def test_gemm_rowcol_static_activation_scale_full_size(dev):
+    """The attention projection with a static per-tensor activation scale
+    (the benchmark's static workload: the scale calibrated on the layer's
+    input, then the static quantizer) x per-channel weights, sampled rows."""
+    cfg = workloads.LLAMA_ATTN
+    X = workloads.activations((cfg.M, cfg.K), cfg.x_kind, cfg.seed, device=dev)
+    W = workloads.weights((cfg.N, cfg.K), cfg.seed + 1, device=dev)
+    sx = fg.tensor_scale(X)
+    Xq = fg.quant_static(X, sx)
+    Wq, sw = fg.quant_rows(W)
+    Y = fg.gemm_rowcol(Xq, sx, Wq, sw)
+    fg.check_device_status()
+    rng = np.random.default_rng(2)
+    tiles = np.arange(0, cfg.M, 128)
+    rows = np.unique(np.concatenate([tiles[::2], tiles[1::2] + 127, rng.integers(0, cfg.M, 16)]))
+    Xb = bits16(X)
+    sx_r = np.array([oracle.tensor_scale(Xb)], dtype=np.float32)
+    assert to_np(sx).view(np.uint32)[0] == sx_r.view(np.uint32)[0]
+    Xq_r = oracle.quant_static(Xb[rows], sx_r[0])
+    Wq_r, sw_r = oracle.quant_rows(bits16(W))
+    Y_ref, S = oracle.gemm_rowcol(Xq_r, sx_r, Wq_r, sw_r)
+    assert_gemm_close(y_to_f64(Y[torch.as_tensor(rows, device=dev)]), Y_ref, S, "static per-tensor 4096^3")
+
+
 def test_gemm_rowcol_empty_and_repeatable(dev):
     (Xq, sx, Wq, sw), _ = make_operands(dev, 200, 512, 1024, 0, 0, seed=1)
     Y1 = fg.gemm_rowcol(Xq, sx, Wq, sw)
