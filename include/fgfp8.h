@@ -60,7 +60,7 @@ typedef enum {
   FGFP8_ERR_INVALID_ARG = 1, /* null pointer, bad enum, negative size */
   FGFP8_ERR_SHAPE = 2,       /* K or N not a multiple of 128, ld too small, size too large */
   FGFP8_ERR_ALIGN = 3,       /* a pointer or leading dimension breaks the 16-byte rule */
-  FGFP8_ERR_UNSUPPORTED = 4, /* a valid request this build does not implement */
+  FGFP8_ERR_UNSUPPORTED = 4, /* a valid request the library does not implement */
   FGFP8_ERR_CUDA = 5,        /* a CUDA runtime or driver call failed */
   FGFP8_ERR_TIMEOUT = 6,     /* a kernel gave up on a barrier wait (device status) */
   FGFP8_ERR_DEVICE = 7       /* a kernel rejected its device-side inputs (device status) */
