@@ -156,6 +156,62 @@ def test_quant_weight_small(dev, fmt, N, K):
     assert_scales_equal(to_np(Ws), Ws_ref, "weight scales")
 
 
+def special_blocks():
+    """A [256, 512] bf16 weight whose eight 128x128 blocks each hold one
+    degenerate pattern: all zero, negative zero, rounding ties, near the bf16
+    maximum, bf16 subnormals, below the amax floor, a ramp, and a single
+    nonzero element."""
+    W = torch.zeros((256, 512))
+    blocks = [(r, c) for r in range(2) for c in range(4)]
+    def blk(i):
+        r, c = blocks[i]
+        return W[r * 128:(r + 1) * 128, c * 128:(c + 1) * 128]
+    blk(1)[5, 7] = -0.0
+    b = blk(2); b[0, 0] = 448; b[0, 1] = 17; b[0, 2] = 19; b[1, 0] = 1.0625; b[1, 1] = -17
+    b = blk(3); b[0, 0] = 3.3895e38; b[0, 1] = -1e38; b[2, 2] = 1.0
+    blk(4).fill_(9.1835e-41); blk(4)[3, 3] = -9.1835e-41
+    b = blk(5); b[0, 0] = 5e-5; b[9, 9] = -2.5e-5
+    blk(6).copy_(torch.linspace(-1, 1, 128 * 128).reshape(128, 128))
+    blk(7)[64, 64] = -0.75
+    return W.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("fmt", [F32, UE8M0])
+def test_quant_weight_special_blocks(dev, fmt):
+    W = special_blocks()
+    W = torch.cat([W, -W], dim=0)
+    Wq, Ws = fg.quant_weight(W.to(dev), fmt)
+    Wq_ref, Ws_ref = oracle.quant_weight(bits16(W), fmt)
+    assert_codes_equal(to_np(Wq), Wq_ref, "special weight codes")
+    assert_scales_equal(to_np(Ws), Ws_ref, "special weight scales")
+    assert to_np(Wq)[5, 128 + 7] == 0x80                 # negative zero keeps its sign
+
+
+@pytest.mark.parametrize("fmt", [F32, UE8M0])
+def test_quant_weight_nonfinite_blocks(dev, fmt):
+    """Finite blocks stay bit-exact next to blocks holding NaN or Inf, whose
+    scale is non-finite (their codes are unspecified)."""
+    W = workloads.weights((256, 384), seed=4)
+    W[3, 5] = float("nan")                               # block (0, 0)
+    W[200, 300] = float("inf")                           # block (1, 2)
+    W[130, 140] = float("-inf")                          # block (1, 1)
+    Wq, Ws = fg.quant_weight(W.to(dev), fmt)
+    Wq_ref, Ws_ref = oracle.quant_weight(bits16(W), fmt)
+    Wq, Ws = to_np(Wq), to_np(Ws)
+    bad = {(0, 0), (1, 2), (1, 1)}
+    for nb in range(2):
+        for kb in range(3):
+            rows, cols = slice(nb * 128, nb * 128 + 128), slice(kb * 128, kb * 128 + 128)
+            if (nb, kb) in bad:
+                if fmt == F32:
+                    assert not np.isfinite(Ws[nb, kb])
+                else:
+                    assert Ws[nb, kb] == 0xFF
+            else:
+                assert_codes_equal(Wq[rows, cols], Wq_ref[rows, cols], "finite block")
+                assert_scales_equal(Ws[nb:nb + 1, kb:kb + 1], Ws_ref[nb:nb + 1, kb:kb + 1], "finite block scale")
+
+
 @pytest.mark.parametrize("fmt", [F32, UE8M0])
 def test_quant_weight_strided(dev, fmt):
     N, K = 256, 384

@@ -36,6 +36,39 @@ def test_quant_rows(dev, R, K, kind):
     assert_scales_equal(to_np(s), s_r, f"row scales {R}x{K}")
 
 
+@pytest.mark.parametrize("K", [256, 8192])
+def test_quant_rows_special_values(dev, K):
+    """Degenerate rows (all zero, negative zero, ties, near the bf16 maximum,
+    subnormals, below the amax floor) bit-exact, for both row kernels (one
+    warp per row up to 4096 elements, one CTA per row above); rows holding
+    NaN or Inf get a non-finite scale while the other rows stay exact."""
+    z = torch.zeros(K)
+    rows = [z.clone()]
+    r = z.clone(); r[3] = -0.0; rows.append(r)
+    r = z.clone(); r[0] = 448; r[1] = 17; r[2] = 19; r[K - 1] = 1.0625; r[K // 2] = -17; rows.append(r)
+    r = z.clone(); r[0] = 3.3895e38; r[K - 2] = -1e38; r[2] = 1.0; rows.append(r)
+    r = torch.full((K,), 9.1835e-41); r[5] = -9.1835e-41; rows.append(r)
+    r = z.clone(); r[0] = 5e-5; r[K - 1] = -2.5e-5; rows.append(r)
+    r = torch.linspace(-1, 1, K); rows.append(r)
+    X = torch.stack(rows).to(torch.bfloat16)
+    X = torch.cat([X, -X], dim=0)
+    Xq, s = fg.quant_rows(X.to(dev))
+    fg.check_device_status()
+    Xq_r, s_r = oracle.quant_rows(bits16(X))
+    assert_codes_equal(to_np(Xq), Xq_r, f"special rows K={K}")
+    assert_scales_equal(to_np(s), s_r, f"special row scales K={K}")
+    assert to_np(Xq)[1, 3] == 0x80
+    Y = X.clone()
+    Y[2, K - 1] = float("nan")
+    Y[5, 0] = float("inf")
+    Yq, sy = fg.quant_rows(Y.to(dev))
+    sy = to_np(sy)
+    assert not np.isfinite(sy[2]) and not np.isfinite(sy[5])
+    ok = [i for i in range(Y.shape[0]) if i not in (2, 5)]
+    assert_codes_equal(to_np(Yq)[ok], Xq_r[ok], "finite rows next to non-finite ones")
+    assert_scales_equal(sy[ok], s_r[ok], "finite row scales")
+
+
 def test_quant_rows_strided_input(dev):
     R, K, ldx = 20, 1024, 1536
     big = workloads.activations((R, ldx), "normal_outliers", seed=9).to(dev)
