@@ -64,7 +64,7 @@ WORKLOAD_ALIASES = {
     "llama_attn": workloads.LLAMA_ATTN.name, "tiny": workloads.TINY.name,
     "llama_gate_up": workloads.LLAMA_GATE_UP.name, "llama_down": workloads.LLAMA_DOWN.name,
     **{f"ds_decode_m{m}": workloads.DS_DECODE[m].name for m in (1, 8, 32, 64)},
-    "moe": workloads.MOE.name, "moe_small": workloads.MOE_SMALL.name,
+    "moe": workloads.MOE.name, "moe_small": workloads.MOE_SMALL.name, "moe_fp32": workloads.MOE_F32.name,
     "llama_attn_dynamic": f"{workloads.LLAMA_ATTN.name}_fp8_dynamic",
     "llama_attn_static": f"{workloads.LLAMA_ATTN.name}_static_tensor",
     "llama_gate_up_dynamic": f"{workloads.LLAMA_GATE_UP.name}_fp8_dynamic",
@@ -553,7 +553,7 @@ def make_layer(name, dev, tokens=None):
     if name in ROWCOL:
         cfg, scheme = ROWCOL[name]
         return RowColLayer(cfg, scheme, dev)
-    for cfg in (workloads.MOE, workloads.MOE_SMALL):
+    for cfg in (workloads.MOE, workloads.MOE_SMALL, workloads.MOE_F32):
         if name == cfg.name:
             return MoELayer(cfg, dev)
     return DenseLayer(workloads.LINEARS[name], dev)
@@ -720,7 +720,7 @@ class OracleSample:
             self.desc = (f"first {self.rows} of {cfg.M} rows x the full [{cfg.N}, {cfg.K}] weight, "
                          f"{self.scheme} scales")
             return
-        moe = {c.name: c for c in (workloads.MOE, workloads.MOE_SMALL, workloads.MOE_DECODE,
+        moe = {c.name: c for c in (workloads.MOE, workloads.MOE_SMALL, workloads.MOE_F32, workloads.MOE_DECODE,
                                    workloads.MOE_DECODE_SMALL)}
         if name in moe:
             cfg = moe[name]

@@ -66,6 +66,8 @@ MOE = MoE("deepseek_v3_moe_256x4096x7168_top8")
 # the same expert shapes with 32 experts and 512 tokens (~1 GB of weights): a
 # profiling case larger than L2 but small enough for multi-pass captures
 MOE_SMALL = MoE("deepseek_v3_moe_32x4096x7168_top8_512tok", E=32, tokens=512)
+# the expert layer with fp32 block scales (the promotion kernel's grouped path)
+MOE_F32 = replace(MOE, name="deepseek_v3_moe_256x4096x7168_top8_fp32", fmt=SCALE_F32)
 # decode step of the same expert layer: 128 tokens, top-8, in the masked
 # layout (every expert a fixed block of 128 rows, its first counts[e] used)
 MOE_DECODE = MoE("deepseek_v3_moe_decode_masked_256x4096x7168_top8_128tok", tokens=128)
