@@ -44,6 +44,7 @@ SIGNATURES = {
     "fgfp8_gemm_swiglu_quant": (_INT, [_P, _P, _I64, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]),
     "fgfp8_masked_gemm": (_INT, [_P, _P, _I64, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _INT, _P]),
     "fgfp8_check_device_status": (_INT, [_P]),
+    "fgfp8_selftest_expired_wait": (_INT, [_P]),
 }
 
 _lock = threading.Lock()
@@ -109,6 +110,7 @@ fgfp8_gemm_rowcol = _raw("fgfp8_gemm_rowcol")
 fgfp8_gemm_swiglu_quant = _raw("fgfp8_gemm_swiglu_quant")
 fgfp8_masked_gemm = _raw("fgfp8_masked_gemm")
 fgfp8_check_device_status = _raw("fgfp8_check_device_status")
+fgfp8_selftest_expired_wait = _raw("fgfp8_selftest_expired_wait")
 
 
 def fgfp8_last_error_string() -> str:
@@ -329,6 +331,12 @@ def gemm_swiglu_quant(Xq, Xs, Wq_gu, Ws_gu, Hq=None, Hs=None, ld_h: int | None =
                                    Hq.data_ptr(), Hs.data_ptr(), ld_h, M, I, K, _stream(stream)),
            "fgfp8_gemm_swiglu_quant")
     return Hq, Hs
+
+
+def selftest_expired_wait(stream=None) -> None:
+    """Launch the bounded-wait self-test (a wait that nothing completes; it
+    gives up after one second and records a timeout in the status word)."""
+    _check(fgfp8_selftest_expired_wait(_stream(stream)), "fgfp8_selftest_expired_wait")
 
 
 def check_device_status(stream=None) -> None:

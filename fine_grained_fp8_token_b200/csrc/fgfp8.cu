@@ -782,6 +782,15 @@ fgfp8_status fgfp8_gemm_swiglu_quant(const uint8_t* Xq, const float* Xs, int64_t
                                                Hs, ld_h);
 }
 
+fgfp8_status fgfp8_selftest_expired_wait(void* stream) {
+  int dev;
+  DeviceInfo info;
+  fgfp8_status st = current_device(&dev, &info);
+  if (st != FGFP8_OK) return st;
+  fgfp8::selftest_expired_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
+  return check_launch("self-test launch");
+}
+
 fgfp8_status fgfp8_check_device_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
@@ -799,6 +808,8 @@ fgfp8_status fgfp8_check_device_status(void* stream) {
       return fail(FGFP8_ERR_TIMEOUT, "a GEMM MMA wait exceeded its limit");
     case fgfp8::kDevTimeoutEpilogue:
       return fail(FGFP8_ERR_TIMEOUT, "a GEMM epilogue wait exceeded its limit");
+    case fgfp8::kDevTimeoutSelftest:
+      return fail(FGFP8_ERR_TIMEOUT, "the bounded-wait self-test's wait expired");
     case fgfp8::kDevBadGroupOffsets:
       return fail(FGFP8_ERR_DEVICE, "group_offs is inconsistent (not a non-decreasing 0..M_total cover)");
     default:

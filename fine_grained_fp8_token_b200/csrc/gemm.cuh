@@ -42,6 +42,18 @@ __device__ int g_device_status;
 
 __device__ __forceinline__ void record_status(int code) { atomicCAS(&g_device_status, 0, code); }
 
+// Self-test of the bounded waits: one thread waits on an mbarrier that
+// nothing completes.  The wait gives up after its limit, the status word
+// records it and the kernel exits, so the context stays usable.
+__global__ void selftest_expired_wait_kernel() {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbarrier_init();
+    if (!mbar_wait(&bar, 0)) record_status(kDevTimeoutSelftest);
+  }
+}
+
 // Tile configuration of the dense / grouped kernel.  BN: output columns per
 // tile; CW: columns per promotion warp (each warp owns 32 rows x CW columns).
 template <int BN, int CW>

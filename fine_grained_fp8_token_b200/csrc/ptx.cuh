@@ -15,6 +15,7 @@ enum : int {
   kDevTimeoutMma = 2,
   kDevTimeoutEpilogue = 3,
   kDevBadGroupOffsets = 4,
+  kDevTimeoutSelftest = 5,
 };
 
 // Upper bound on any single barrier wait.  A healthy wait here lasts at most

@@ -302,6 +302,16 @@ fgfp8_status fgfp8_linear_noalloc(const void* X, int64_t ldx, const uint8_t* Wq,
                                   int64_t N, int64_t K, int fmt, void* stream);
 
 /*
+ * Diagnostic with no counterpart on the pages: a self-test of the kernels'
+ * bounded barrier waits.  Launches one thread on `stream` that waits on a
+ * barrier nothing completes; after the one-second limit the wait gives up,
+ * the device status word records a timeout and the kernel exits.
+ * fgfp8_check_device_status then returns FGFP8_ERR_TIMEOUT, and the context
+ * stays usable.  Returns FGFP8_ERR_CUDA without an sm_100a device.
+ */
+fgfp8_status fgfp8_selftest_expired_wait(void* stream);
+
+/*
  * Synchronizes `stream`, then reads and clears the device status word that
  * the kernels set when they give up.  It returns FGFP8_OK,
  * FGFP8_ERR_TIMEOUT (a barrier wait ran past its one-second limit),

@@ -162,5 +162,6 @@ def test_valid_call_without_gpu_fails_loudly():
     assert fg.fgfp8_linear(A, 256, A, A, 4, A, A, A, 4, 256, 256, 0, None) == CUDA
     assert fg.fgfp8_quant_rows(A, 4, 256, 256, A, A, None) == CUDA
     assert fg.fgfp8_gemm_rowcol(A, A, 0, A, A, 0, A, 4, 256, 256, None) == CUDA
+    assert fg.fgfp8_selftest_expired_wait(None) == CUDA
     with pytest.raises(fg.FGFP8Error):
         fg._check(fg.fgfp8_quant_weight(A, 128, 256, 256, A, A, 0, None), "quant_weight")
