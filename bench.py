@@ -403,10 +403,10 @@ class MLPLayer:
 class MaskedMoELayer:
     """Decode step of the expert layer in the masked layout: 128 tokens
     routed top-8 (Zipf-skewed) to 256 experts, every expert a fixed block of
-    cap = 128 rows of which the first counts[e] hold tokens; the step is the
-    1x128 quantizer over the whole [E * cap, K] buffer and fgfp8_masked_gemm.
-    Experts without tokens are skipped, so the GEMM streams the weights of
-    the active experts only."""
+    cap = 128 rows of which the first counts[e] hold tokens; the step is
+    fgfp8_masked_linear: the 1x128 quantizer over the token rows only, then
+    the masked GEMM as its programmatic dependent.  Experts without tokens
+    are skipped, so the GEMM streams the weights of the active experts only."""
 
     CAP = 128
 
@@ -433,23 +433,26 @@ class MaskedMoELayer:
         self.fg.quant_weight(self.W, self.cfg.fmt, Wq=self.Wq[0], Ws=self.Ws[0])
 
     def quant_act(self, X=None):
-        self.fg.quant_act(self.X if X is None else X, self.cfg.fmt, Xq=self.Xq, Xs=self.Xs, ld_s=self.ld_s)
+        # the token rows only: padding rows are never read by the masked GEMM
+        self.fg.quant_act_masked(self.X if X is None else X, self.counts, self.cfg.E, self.cfg.fmt, Xq=self.Xq,
+                                 Xs=self.Xs, ld_s=self.ld_s)
 
     def gemm(self):
         self.fg.masked_gemm(self.Xq, self.Xs, self.Wq, self.Ws, self.counts, self.cfg.fmt, Y=self.Y)
 
     def linear(self, X=None):
-        self.quant_act(X)
-        self.gemm()
+        self.fg.masked_linear(self.X if X is None else X, self.Wq, self.Ws, self.counts, self.cfg.fmt, Y=self.Y,
+                              Xq=self.Xq, Xs=self.Xs, ld_s=self.ld_s)
 
     def flops(self):
         c = self.cfg
         return 2.0 * float(self.r.counts.sum()) * c.N * c.K
 
     def act_bytes(self):
+        # the token rows read and their codes and scales written
         c = self.cfg
-        M = c.E * self.CAP
-        return 3.0 * M * c.K + (4 if c.fmt == 0 else 1) * M * c.K / 128
+        rows = float(self.r.counts.sum())
+        return 3.0 * rows * c.K + (4 if c.fmt == 0 else 1) * rows * c.K / 128
 
     def gemm_bytes(self):
         # the active experts' weights and scales, the token rows' codes and scales, Y's token rows
@@ -898,7 +901,7 @@ def main():
             "apart_sum_us": 1e3 * (r["quant_ms"] + r["gemm_ms"]),
         },
         "step_call": ("fgfp8_quant_act + fgfp8_gemm_swiglu_quant + fgfp8_gemm" if isinstance(layer, MLPLayer) else
-                      "fgfp8_quant_act + fgfp8_masked_gemm" if isinstance(layer, MaskedMoELayer) else
+                      "fgfp8_masked_linear" if isinstance(layer, MaskedMoELayer) else
                       "fgfp8_grouped_linear" if isinstance(layer, MoELayer) else
                       ("fgfp8_quant_rows + fgfp8_gemm_rowcol" if getattr(layer, "scheme", None) == "fp8_dynamic"
                        else "fgfp8_quant_static + fgfp8_gemm_rowcol") if isinstance(layer, RowColLayer)

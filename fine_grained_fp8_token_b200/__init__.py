@@ -43,6 +43,8 @@ SIGNATURES = {
     "fgfp8_gemm_rowcol": (_INT, [_P, _P, _INT, _P, _P, _INT, _P, _I64, _I64, _I64, _P]),
     "fgfp8_gemm_swiglu_quant": (_INT, [_P, _P, _I64, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]),
     "fgfp8_masked_gemm": (_INT, [_P, _P, _I64, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _INT, _P]),
+    "fgfp8_quant_act_masked": (_INT, [_P, _I64, _P, _I32, _I64, _I64, _P, _P, _I64, _INT, _P]),
+    "fgfp8_masked_linear": (_INT, [_P, _I64, _P, _P, _I64, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _INT, _P]),
     "fgfp8_check_device_status": (_INT, [_P]),
     "fgfp8_selftest_expired_wait": (_INT, [_P]),
 }
@@ -109,6 +111,8 @@ fgfp8_quant_static = _raw("fgfp8_quant_static")
 fgfp8_gemm_rowcol = _raw("fgfp8_gemm_rowcol")
 fgfp8_gemm_swiglu_quant = _raw("fgfp8_gemm_swiglu_quant")
 fgfp8_masked_gemm = _raw("fgfp8_masked_gemm")
+fgfp8_quant_act_masked = _raw("fgfp8_quant_act_masked")
+fgfp8_masked_linear = _raw("fgfp8_masked_linear")
 fgfp8_check_device_status = _raw("fgfp8_check_device_status")
 fgfp8_selftest_expired_wait = _raw("fgfp8_selftest_expired_wait")
 
@@ -298,6 +302,44 @@ def masked_gemm(Xq, Xs, Wq, Ws, counts, fmt: int, Y=None, stream=None):
         Y = torch.empty((M_total, N), dtype=torch.bfloat16, device=Xq.device)
     _check(fgfp8_masked_gemm(Xq.data_ptr(), Xs.data_ptr(), Xs.shape[1], Wq.data_ptr(), Ws.data_ptr(), Y.data_ptr(),
                              counts.data_ptr(), E, cap, N, K, fmt, _stream(stream)), "fgfp8_masked_gemm")
+    return Y
+
+
+def quant_act_masked(X, counts, E: int, fmt: int, Xq=None, Xs=None, ld_s: int | None = None, stream=None):
+    """The 1x128 quantizer over the token rows of the masked layout only
+    (X bf16 [E * cap, K]; expert e's tokens in rows [e * cap, e * cap +
+    counts[e]), counts int32 [E] on the device).  Padding rows of Xq / Xs
+    are left as they are.  Returns (Xq, Xs)."""
+    import torch
+    M, K = X.shape
+    cap = M // E
+    ld_s = scale_rows(M, fmt) if ld_s is None else ld_s
+    if Xq is None:
+        Xq = torch.empty((M, K), dtype=torch.uint8, device=X.device)
+    if Xs is None:
+        Xs = torch.empty((K // 128, ld_s), dtype=torch.float32 if fmt == SCALE_F32 else torch.uint8, device=X.device)
+    _check(fgfp8_quant_act_masked(X.data_ptr(), X.stride(0), counts.data_ptr(), E, cap, K, Xq.data_ptr(),
+                                  Xs.data_ptr(), ld_s, fmt, _stream(stream)), "fgfp8_quant_act_masked")
+    return Xq, Xs
+
+
+def masked_linear(X, Wq, Ws, counts, fmt: int, Y=None, Xq=None, Xs=None, ld_s: int | None = None, stream=None):
+    """The masked expert layer in one call (token rows quantized, then the
+    masked GEMM).  Returns Y bf16 [E * cap, N] (padding rows not written)."""
+    import torch
+    M, K = X.shape
+    E, N, _ = Wq.shape
+    cap = M // E
+    ld_s = scale_rows(M, fmt) if ld_s is None else ld_s
+    if Xq is None:
+        Xq = torch.empty((M, K), dtype=torch.uint8, device=X.device)
+    if Xs is None:
+        Xs = torch.empty((K // 128, ld_s), dtype=torch.float32 if fmt == SCALE_F32 else torch.uint8, device=X.device)
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _check(fgfp8_masked_linear(X.data_ptr(), X.stride(0), Xq.data_ptr(), Xs.data_ptr(), ld_s, Wq.data_ptr(),
+                               Ws.data_ptr(), Y.data_ptr(), counts.data_ptr(), E, cap, N, K, fmt, _stream(stream)),
+           "fgfp8_masked_linear")
     return Y
 
 

@@ -526,6 +526,68 @@ fgfp8_status noalloc_scratch(int dev, uint8_t** out) {
   return FGFP8_OK;
 }
 
+// Masked expert GEMM; with dry set, only validates.
+fgfp8_status masked_impl(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws, void* Y,
+                         const int32_t* counts, int32_t E, int64_t cap, int64_t N, int64_t K, int fmt, void* stream,
+                         bool dry) {
+  if (E <= 0) return fail(FGFP8_ERR_INVALID_ARG, "E must be >= 1");
+  if (cap <= 0 || cap % 128 != 0) return fail(FGFP8_ERR_SHAPE, "cap must be a positive multiple of 128");
+  if (static_cast<int64_t>(E) * cap >= (int64_t(1) << 31)) return fail(FGFP8_ERR_SHAPE, "E*cap must be < 2^31");
+  const int64_t M_total = static_cast<int64_t>(E) * cap;
+  fgfp8_status st = check_gemm_common(Xq, Xs, ld_s, Wq, Ws, Y, M_total, N, K, fmt);
+  if (st != FGFP8_OK) return st;
+  if (!counts) return fail(FGFP8_ERR_INVALID_ARG, "counts is NULL");
+  if (!aligned(counts, 4)) return fail(FGFP8_ERR_ALIGN, "counts must be 4-byte aligned");
+  if (static_cast<int64_t>(E) * N >= (int64_t(1) << 31)) return fail(FGFP8_ERR_SHAPE, "E*N must be < 2^31");
+  if (dry) return FGFP8_OK;
+  int dev;
+  DeviceInfo info;
+  st = current_device(&dev, &info);
+  if (st != FGFP8_OK) return st;
+  return dispatch_gemm<true>(Xq, Xs, ld_s, Wq, Ws, Y, M_total, N, K, fmt, counts, E, static_cast<int64_t>(E) * N,
+                             reinterpret_cast<cudaStream_t>(stream), dev, info.sm_count, 0, static_cast<int>(cap));
+}
+
+// Activation quantizer over the token rows of the masked layout; with dry
+// set, only validates.
+fgfp8_status quant_act_masked_impl(const void* X, int64_t ldx, const int32_t* counts, int32_t E, int64_t cap,
+                                   int64_t K, uint8_t* Xq, void* Xs, int64_t ld_s, int fmt, void* stream, bool dry) {
+  if (E <= 0) return fail(FGFP8_ERR_INVALID_ARG, "E must be >= 1");
+  if (cap <= 0 || cap % 128 != 0) return fail(FGFP8_ERR_SHAPE, "cap must be a positive multiple of 128");
+  if (static_cast<int64_t>(E) * cap >= (int64_t(1) << 31)) return fail(FGFP8_ERR_SHAPE, "E*cap must be < 2^31");
+  if (E > 65535) return fail(FGFP8_ERR_SHAPE, "E must be <= 65535");
+  if (!counts) return fail(FGFP8_ERR_INVALID_ARG, "counts is NULL");
+  if (!aligned(counts, 4)) return fail(FGFP8_ERR_ALIGN, "counts must be 4-byte aligned");
+  const int64_t M = static_cast<int64_t>(E) * cap;
+  // the same checks as the quantizer over all E * cap rows
+  fgfp8_status st = quant_act_impl(X, M, K, ldx, Xq, Xs, ld_s, fmt, stream, true);
+  if (st != FGFP8_OK) return st;
+  if (dry) return FGFP8_OK;
+  int dev;
+  DeviceInfo info;
+  st = current_device(&dev, &info);
+  if (st != FGFP8_OK) return st;
+  // blocks per expert: a full expert block in about seven passes of 32
+  // groups each; blocks beyond an expert's count exit at once
+  const int64_t most = cap * (K / 128);                       // groups of a full expert block
+  int64_t bx = (most + 255) / 256;
+  bx = bx < 1 ? 1 : (bx > 32 ? 32 : bx);
+  const dim3 grid(static_cast<unsigned>(bx), static_cast<unsigned>(E));
+  fgfp8::FastDiv kbd(static_cast<uint32_t>(K / 128));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (fmt == FGFP8_SCALE_F32)
+    fgfp8::quant_act_masked_kernel<0><<<grid, 256, 0, s>>>(reinterpret_cast<const uint16_t*>(X), counts,
+                                                           static_cast<uint32_t>(cap), static_cast<uint32_t>(K),
+                                                           static_cast<uint64_t>(ldx), Xq, Xs,
+                                                           static_cast<uint64_t>(ld_s), kbd);
+  else
+    fgfp8::quant_act_masked_kernel<1><<<grid, 256, 0, s>>>(reinterpret_cast<const uint16_t*>(X), counts,
+                                                           static_cast<uint32_t>(cap), static_cast<uint32_t>(K),
+                                                           static_cast<uint64_t>(ldx), Xq, Xs,
+                                                           static_cast<uint64_t>(ld_s), kbd);
+  return check_launch("masked quant_act launch");
+}
+
 }  // namespace
 
 extern "C" {
@@ -746,21 +808,24 @@ fgfp8_status fgfp8_gemm_rowcol(const uint8_t* Xq, const float* sx, int x_per_ten
 fgfp8_status fgfp8_masked_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
                                void* Y, const int32_t* counts, int32_t E, int64_t cap, int64_t N, int64_t K, int fmt,
                                void* stream) {
-  if (E <= 0) return fail(FGFP8_ERR_INVALID_ARG, "E must be >= 1");
-  if (cap <= 0 || cap % 128 != 0) return fail(FGFP8_ERR_SHAPE, "cap must be a positive multiple of 128");
-  if (static_cast<int64_t>(E) * cap >= (int64_t(1) << 31)) return fail(FGFP8_ERR_SHAPE, "E*cap must be < 2^31");
-  const int64_t M_total = static_cast<int64_t>(E) * cap;
-  fgfp8_status st = check_gemm_common(Xq, Xs, ld_s, Wq, Ws, Y, M_total, N, K, fmt);
+  return masked_impl(Xq, Xs, ld_s, Wq, Ws, Y, counts, E, cap, N, K, fmt, stream, false);
+}
+
+fgfp8_status fgfp8_quant_act_masked(const void* X, int64_t ldx, const int32_t* counts, int32_t E, int64_t cap,
+                                    int64_t K, uint8_t* Xq, void* Xs, int64_t ld_s, int fmt, void* stream) {
+  return quant_act_masked_impl(X, ldx, counts, E, cap, K, Xq, Xs, ld_s, fmt, stream, false);
+}
+
+fgfp8_status fgfp8_masked_linear(const void* X, int64_t ldx, uint8_t* Xq, void* Xs, int64_t ld_s, const uint8_t* Wq,
+                                 const void* Ws, void* Y, const int32_t* counts, int32_t E, int64_t cap, int64_t N,
+                                 int64_t K, int fmt, void* stream) {
+  fgfp8_status st = quant_act_masked_impl(X, ldx, counts, E, cap, K, Xq, Xs, ld_s, fmt, stream, true);
   if (st != FGFP8_OK) return st;
-  if (!counts) return fail(FGFP8_ERR_INVALID_ARG, "counts is NULL");
-  if (!aligned(counts, 4)) return fail(FGFP8_ERR_ALIGN, "counts must be 4-byte aligned");
-  if (static_cast<int64_t>(E) * N >= (int64_t(1) << 31)) return fail(FGFP8_ERR_SHAPE, "E*N must be < 2^31");
-  int dev;
-  DeviceInfo info;
-  st = current_device(&dev, &info);
+  st = masked_impl(Xq, Xs, ld_s, Wq, Ws, Y, counts, E, cap, N, K, fmt, stream, true);
   if (st != FGFP8_OK) return st;
-  return dispatch_gemm<true>(Xq, Xs, ld_s, Wq, Ws, Y, M_total, N, K, fmt, counts, E, static_cast<int64_t>(E) * N,
-                             reinterpret_cast<cudaStream_t>(stream), dev, info.sm_count, 0, static_cast<int>(cap));
+  st = quant_act_masked_impl(X, ldx, counts, E, cap, K, Xq, Xs, ld_s, fmt, stream, false);
+  if (st != FGFP8_OK) return st;
+  return masked_impl(Xq, Xs, ld_s, Wq, Ws, Y, counts, E, cap, N, K, fmt, stream, false);
 }
 
 fgfp8_status fgfp8_gemm_swiglu_quant(const uint8_t* Xq, const float* Xs, int64_t ld_s, const uint8_t* Wq_gu,

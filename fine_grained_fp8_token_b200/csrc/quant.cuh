@@ -189,6 +189,52 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
 }
 
 // ---------------------------------------------------------------------------
+// Activation quantization in the masked expert layout: expert e's tokens are
+// rows [e * cap, e * cap + counts[e]) of X; only those rows are quantized
+// (the padding rows' codes and scales are left as they are, and the masked
+// GEMM never reads them).  blockIdx.y = expert; the blocks of an expert
+// stride over its count * K/128 groups, 8 lanes per group as above.  A
+// count outside [0, cap] is clamped to it here; the masked GEMM reports it.
+// ---------------------------------------------------------------------------
+template <int FMT>
+__global__ void __launch_bounds__(256) quant_act_masked_kernel(const uint16_t* __restrict__ X,
+                                                               const int32_t* __restrict__ counts, uint32_t cap,
+                                                               uint32_t K, uint64_t ldx, uint8_t* __restrict__ Xq,
+                                                               void* __restrict__ Xs, uint64_t ld_s, FastDiv kb_div) {
+  griddep_launch_dependents();
+  const uint32_t e = blockIdx.y;
+  const int32_t c = __ldg(counts + e);
+  const uint32_t rows = c <= 0 ? 0u : (static_cast<uint32_t>(c) < cap ? static_cast<uint32_t>(c) : cap);
+  const uint32_t total = rows * kb_div.d;
+  const uint32_t lane = threadIdx.x & 31u;
+  const uint32_t sub = lane & 7u;
+  const uint32_t gmask = 0xFFu << (lane & 24u);
+  const uint32_t row0 = e * cap;
+  for (uint32_t gi = (blockIdx.x * blockDim.x + threadIdx.x) >> 3; gi < total; gi += (gridDim.x * blockDim.x) >> 3) {
+    const uint32_t r = kb_div.div(gi);
+    const uint32_t g = gi - r * kb_div.d;
+    const uint32_t m = row0 + r;
+    const uint16_t* src = X + m * ldx + g * kGroup + sub * 16u;
+    const uint4 v0 = ld_stream_v4(src), v1 = ld_stream_v4(src + 8);
+    uint32_t a = max(absmax_bits8(v0), absmax_bits8(v1));
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) a = max(a, __shfl_xor_sync(gmask, a, o));
+    const GroupScale gs = make_scale<FMT>(a);
+    uint4 codes;
+    codes.x = quant4<FMT>(v0.x, v0.y, gs);
+    codes.y = quant4<FMT>(v0.z, v0.w, gs);
+    codes.z = quant4<FMT>(v1.x, v1.y, gs);
+    codes.w = quant4<FMT>(v1.z, v1.w, gs);
+    *reinterpret_cast<uint4*>(Xq + static_cast<uint64_t>(m) * K + g * kGroup + sub * 16u) = codes;
+    if (sub == 0) {
+      const uint64_t si = static_cast<uint64_t>(g) * ld_s + m;
+      if (FMT == 0) reinterpret_cast<float*>(Xs)[si] = gs.s;
+      else reinterpret_cast<uint8_t*>(Xs)[si] = static_cast<uint8_t>(gs.e8);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Weight quantization.  One 256-thread CTA per 128x128 block: half-warp h
 // owns rows h, h+16, ..., h+112 of the block; every thread keeps its eight
 // 16-byte chunks in registers across the block-wide amax reduction.

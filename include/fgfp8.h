@@ -159,6 +159,32 @@ fgfp8_status fgfp8_masked_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, 
                                void* stream);
 
 /*
+ * The dynamic 1x128 activation quantizer of fgfp8_quant_act over the token
+ * rows of the masked layout only: rows [e*cap, e*cap + counts[e]) of X for
+ * every expert e.  Padding rows are not read, and their codes and scales
+ * are left as they are (fgfp8_masked_gemm never reads them).
+ *   X        DEVICE bf16 [E*cap, K], row stride ldx; Xq, Xs, ld_s as for
+ *            fgfp8_quant_act with M = E*cap.
+ *   counts   DEVICE int32 [E]; a count below 0 quantizes no row and one
+ *            above cap quantizes cap rows (fgfp8_masked_gemm reports such
+ *            a count).
+ * cap % 128 == 0, 1 <= E <= 65535; the other checks are those of
+ * fgfp8_quant_act.  No counterpart on the pages: the decode step would
+ * otherwise quantize every padding row.
+ */
+fgfp8_status fgfp8_quant_act_masked(const void* X, int64_t ldx, const int32_t* counts, int32_t E, int64_t cap,
+                                    int64_t K, uint8_t* Xq, void* Xs, int64_t ld_s, int fmt, void* stream);
+
+/*
+ * The masked expert layer in one call: fgfp8_quant_act_masked into the
+ * caller's Xq / Xs, then fgfp8_masked_gemm launched as the quantizer's
+ * programmatic dependent.  Every argument is checked before either launch.
+ */
+fgfp8_status fgfp8_masked_linear(const void* X, int64_t ldx, uint8_t* Xq, void* Xs, int64_t ld_s, const uint8_t* Wq,
+                                 const void* Ws, void* Y, const int32_t* counts, int32_t E, int64_t cap, int64_t N,
+                                 int64_t K, int fmt, void* stream);
+
+/*
  * The whole W8A8 linear layer: fgfp8_quant_act of X into the caller's Xq /
  * Xs buffers followed by fgfp8_gemm ("Fine-grained FP8", introduction and
  * "DeepGEMM fast path": activations are quantized on the fly, weights are

@@ -163,5 +163,26 @@ def test_valid_call_without_gpu_fails_loudly():
     assert fg.fgfp8_quant_rows(A, 4, 256, 256, A, A, None) == CUDA
     assert fg.fgfp8_gemm_rowcol(A, A, 0, A, A, 0, A, 4, 256, 256, None) == CUDA
     assert fg.fgfp8_selftest_expired_wait(None) == CUDA
+    assert fg.fgfp8_quant_act_masked(A, 256, A, 2, 128, 256, A, A, 256, 0, None) == CUDA
+    assert fg.fgfp8_masked_linear(A, 256, A, A, 256, A, A, A, A, 2, 128, 256, 256, 0, None) == CUDA
     with pytest.raises(fg.FGFP8Error):
         fg._check(fg.fgfp8_quant_weight(A, 128, 256, 256, A, A, 0, None), "quant_weight")
+
+
+def test_masked_quant_and_linear_validation():
+    """The masked quantizer and the one-call masked layer check their
+    arguments on the host before any launch."""
+    f = fg.fgfp8_quant_act_masked     # X, ldx, counts, E, cap, K, Xq, Xs, ld_s, fmt, stream
+    assert f(A, 256, A, 0, 128, 256, A, A, 256, 0, None) == INVALID          # E < 1
+    assert f(A, 256, A, 2, 100, 256, A, A, 256, 0, None) == SHAPE            # cap % 128
+    assert f(A, 256, A, 70000, 128, 256, A, A, 70000 * 128, 0, None) == SHAPE   # E > 65535
+    assert f(A, 256, 0, 2, 128, 256, A, A, 256, 0, None) == INVALID          # NULL counts
+    assert f(A, 256, A + 2, 2, 128, 256, A, A, 256, 0, None) == ALIGN        # counts alignment
+    assert f(A, 256, A, 2, 128, 200, A, A, 256, 0, None) == SHAPE            # K % 128
+    assert f(A, 256, A, 2, 128, 256, A, A, 128, 0, None) == SHAPE            # ld_s < E * cap
+    assert f(A + 2, 256, A, 2, 128, 256, A, A, 256, 0, None) == ALIGN        # X alignment
+    g = fg.fgfp8_masked_linear        # X, ldx, Xq, Xs, ld_s, Wq, Ws, Y, counts, E, cap, N, K, fmt, stream
+    assert g(A, 256, A, A, 256, A, A, A, A, 2, 128, 200, 256, 0, None) == SHAPE    # N % 128
+    assert g(A, 256, A, A, 256, A, A, A, 0, 2, 128, 256, 256, 0, None) == INVALID  # NULL counts
+    assert g(A, 256, A, A, 256, A, A, A, A, 2, 128, 256, 256, 3, None) == INVALID  # fmt
+

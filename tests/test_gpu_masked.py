@@ -123,3 +123,59 @@ def test_masked_full_decode_step_sampled_experts(dev):
         pad[int(e) * cap:int(e) * cap + int(r.counts[e])] = False
     assert (Y[pad].float() == SENTINEL).all(), "padding rows written"
 
+
+@pytest.mark.parametrize("fmt", [F32, UE8M0])
+def test_quant_act_masked_token_rows_only(dev, fmt):
+    """The masked quantizer writes exactly the token rows, bit-exact with the
+    1x128 quantizer (and the oracle); padding rows (here NaN) are not read
+    and their codes and scales stay as they were.  A count above cap
+    quantizes the whole block."""
+    E, cap, K = 4, 128, 896
+    counts = [5, 0, 128, 77]
+    X = workloads.activations((E * cap, K), "normal_outliers", seed=31)
+    for e, c in enumerate(counts):
+        X[e * cap + c:(e + 1) * cap, ::5] = float("nan")
+    Xd = X.to(dev)
+    Xq_all, Xs_all = fg.quant_act(Xd, fmt)
+    sdt = torch.float32 if fmt == F32 else torch.uint8
+    Xq = torch.full((E * cap, K), 0xAB, dtype=torch.uint8, device=dev)
+    Xs = torch.full(Xs_all.shape, 3, dtype=sdt, device=dev)
+    fg.quant_act_masked(Xd, torch.tensor(counts, dtype=torch.int32, device=dev), E, fmt, Xq=Xq, Xs=Xs)
+    fg.check_device_status()
+    tok = np.concatenate([np.arange(e * cap, e * cap + c) for e, c in enumerate(counts)])
+    pad = np.setdiff1d(np.arange(E * cap), tok)
+    assert torch.equal(Xq[tok], Xq_all[tok])
+    assert torch.equal(Xs[:, tok].contiguous().view(torch.uint8), Xs_all[:, tok].contiguous().view(torch.uint8))
+    Xq_r, Xs_r = oracle.quant_act(bits16(X[tok]), fmt)
+    assert np.array_equal(to_np(Xq[tok]), Xq_r)
+    assert (Xq[pad] == 0xAB).all() and (Xs[:, pad].float() == 3).all()
+    # a count above cap: the whole block is quantized
+    Xq2 = torch.zeros_like(Xq_all)
+    Xs2 = torch.zeros_like(Xs_all)
+    fg.quant_act_masked(Xd, torch.tensor([0, cap + 9, 0, 0], dtype=torch.int32, device=dev), E, fmt, Xq=Xq2, Xs=Xs2)
+    fg.check_device_status()
+    blk = slice(cap, 2 * cap)
+    assert torch.equal(Xq2[blk], Xq_all[blk])
+
+
+@pytest.mark.parametrize("fmt", [F32, UE8M0])
+def test_masked_linear_equals_two_calls(dev, fmt):
+    """fgfp8_masked_linear (token-row quantizer + masked GEMM as its
+    programmatic dependent) gives bit-for-bit the masked quantizer's codes
+    and the masked GEMM's output; token rows also against the oracle."""
+    E, cap, N, K = 5, 128, 256, 512
+    counts = [3, 0, 128, 64, 1]
+    X, W_list, _, _, Wq, Ws = build(dev, E, cap, N, K, fmt, seed=57, counts=counts)
+    Xd = X.to(dev)
+    cnt = torch.tensor(counts, dtype=torch.int32, device=dev)
+    Xq1, Xs1 = fg.quant_act_masked(Xd, cnt, E, fmt)
+    Y1 = torch.full((E * cap, N), SENTINEL, dtype=torch.bfloat16, device=dev)
+    fg.masked_gemm(Xq1, Xs1, Wq, Ws, cnt, fmt, Y=Y1)
+    Y2 = torch.full((E * cap, N), SENTINEL, dtype=torch.bfloat16, device=dev)
+    fg.masked_linear(Xd, Wq, Ws, cnt, fmt, Y=Y2)
+    fg.check_device_status()
+    assert torch.equal(Y1, Y2)
+    check_rows(X, W_list, Y2, counts, cap, fmt, "masked linear")
+    for e, c in enumerate(counts):
+        assert (Y2[e * cap + c:(e + 1) * cap].float() == SENTINEL).all()
+
