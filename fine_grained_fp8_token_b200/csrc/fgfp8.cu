@@ -256,10 +256,7 @@ fgfp8_status dispatch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, cons
   // 128x256 tiles: measured faster per FLOP than 128x128 on B200 even where
   // 128x128 tiles would fill the last wave better (4096^3: 95 us vs 119 us);
   // 128x128 only when N is not a multiple of 256.
-  bool wide = (N % 256 == 0);
-#if defined(FGFP8_FORCE_BN)
-  wide = (FGFP8_FORCE_BN == 256) && (N % 256 == 0);
-#endif
+  const bool wide = (N % 256 == 0);
   constexpr int kWideCW = 128;
   // UE8M0 scales: the tensor core applies them (block-scaled MMA), no promotion.
   if (fmt == FGFP8_SCALE_UE8M0)
@@ -876,7 +873,11 @@ fgfp8_status fgfp8_check_device_status(void* stream) {
     case fgfp8::kDevTimeoutSelftest:
       return fail(FGFP8_ERR_TIMEOUT, "the bounded-wait self-test's wait expired");
     case fgfp8::kDevBadGroupOffsets:
-      return fail(FGFP8_ERR_DEVICE, "group_offs is inconsistent (not a non-decreasing 0..M_total cover)");
+      return fail(FGFP8_ERR_DEVICE,
+                  "group_offs is inconsistent (not a non-decreasing 0..M_total cover) or a masked count is outside "
+                  "[0, cap]");
+    case fgfp8::kDevBadScale:
+      return fail(FGFP8_ERR_DEVICE, "the static quantizer's scale is not positive (<= 0 or NaN)");
     default:
       return fail(FGFP8_ERR_DEVICE, "unknown device status " + std::to_string(v));
   }

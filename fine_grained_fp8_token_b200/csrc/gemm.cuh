@@ -38,10 +38,6 @@
 
 namespace fgfp8 {
 
-__device__ int g_device_status;
-
-__device__ __forceinline__ void record_status(int code) { atomicCAS(&g_device_status, 0, code); }
-
 // Self-test of the bounded waits: one thread waits on an mbarrier that
 // nothing completes.  The wait gives up after its limit, the status word
 // records it and the kernel exits, so the context stays usable.

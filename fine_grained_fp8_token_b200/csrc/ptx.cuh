@@ -16,7 +16,14 @@ enum : int {
   kDevTimeoutEpilogue = 3,
   kDevBadGroupOffsets = 4,
   kDevTimeoutSelftest = 5,
+  kDevBadScale = 6,
 };
+
+// The device status word: the first nonzero code a kernel records stays
+// until fgfp8_check_device_status reads and clears it.
+__device__ int g_device_status;
+
+__device__ __forceinline__ void record_status(int code) { atomicCAS(&g_device_status, 0, code); }
 
 // Upper bound on any single barrier wait.  A healthy wait here lasts at most
 // microseconds; one second means a lost arrival, and the kernel gives up.

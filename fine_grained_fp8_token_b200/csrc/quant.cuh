@@ -20,6 +20,7 @@
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
+#include <cmath>
 #include <cstdint>
 
 #include "ptx.cuh"
@@ -109,20 +110,63 @@ __device__ __forceinline__ float quotient(float x, const GroupScale& g) {
 }
 
 // Four bf16 (two packed words) -> four E4M3 codes in one word (element 0 in
-// the low byte).  Magnitudes are quantized; the four sign bits (bit 7 of the
-// bf16 bytes 1 and 3 of each word) are gathered with one byte permute.
-template <int FMT>
-__device__ __forceinline__ uint32_t quant4(uint32_t w0, uint32_t w1, const GroupScale& g) {
+// the low byte).  Magnitudes are quantized (div(x) = |x| / s); the four sign
+// bits (bit 7 of the bf16 bytes 1 and 3 of each word) are gathered with one
+// byte permute.
+template <typename Div>
+__device__ __forceinline__ uint32_t quant4_by(uint32_t w0, uint32_t w1, const Div& div) {
   const uint32_t c0 = __nv_cvt_float2_to_fp8x2(
-      make_float2(quotient<FMT>(__uint_as_float(w0 << 16), g), quotient<FMT>(__uint_as_float(w0 & 0xFFFF0000u), g)),
-      __NV_SATFINITE, __NV_E4M3);
+      make_float2(div(__uint_as_float(w0 << 16)), div(__uint_as_float(w0 & 0xFFFF0000u))), __NV_SATFINITE, __NV_E4M3);
   const uint32_t c1 = __nv_cvt_float2_to_fp8x2(
-      make_float2(quotient<FMT>(__uint_as_float(w1 << 16), g), quotient<FMT>(__uint_as_float(w1 & 0xFFFF0000u), g)),
-      __NV_SATFINITE, __NV_E4M3);
+      make_float2(div(__uint_as_float(w1 << 16)), div(__uint_as_float(w1 & 0xFFFF0000u))), __NV_SATFINITE, __NV_E4M3);
   const uint32_t codes = __byte_perm(c0, c1, 0x5410);
   const uint32_t signs = __byte_perm(w0, w1, 0x7531) & 0x80808080u;
   return codes | signs;
 }
+
+template <int FMT>
+__device__ __forceinline__ uint32_t quant4(uint32_t w0, uint32_t w1, const GroupScale& g) {
+  return quant4_by(w0, w1, [&g](float x) { return quotient<FMT>(x, g); });
+}
+
+// |x| / s for a caller-given scale s > 0 (static quantization), correctly
+// rounded wherever the E4M3 code depends on it.  Unlike the dynamic scales
+// (amax/448 with |x| <= amax, so the quotient stays below 449), a given scale
+// can meet any bf16 |x|, and the FMA form above fails at the ends of the
+// range: RN(|x| r) overflows to infinity for |x|/s > 2^128 (the correction
+// then gives inf - inf = NaN), and r = RN(1/s) itself overflows or loses
+// precision for s below 2^-126.  So:
+//  * kFast (s in [2^-92, 2^126], checked once per launch): the FMA form.  In
+//    that window 1/s is a normal number, and every quotient >= 2^-11 has
+//    |x| >= 2^-103, so the residual fma(-q0, s, |x|) is exact and Markstein's
+//    theorem gives RN(|x|/s).  Quotients below 2^-11 come out below 2^-10 and
+//    encode to a zero code either way.  When the first approximation q0
+//    reaches 1024 the quotient exceeds 448 and saturates whatever its last
+//    bits: q0 itself is returned (also when it is infinite).
+//  * otherwise: the IEEE quotient (__fdiv_rn) for every element.
+// Host code gets the same operations from the host compiler's IEEE fp32
+// arithmetic, so the host checks run this very function.
+template <bool kFast>
+__host__ __device__ __forceinline__ float static_quotient(float a, float s, float r) {
+#ifdef __CUDA_ARCH__
+  if (kFast) {
+    const float q0 = __fmul_rn(a, r);
+    const float q = __fmaf_rn(__fmaf_rn(-q0, s, a), r, q0);
+    return q0 < 1024.0f ? q : q0;
+  }
+  return __fdiv_rn(a, s);
+#else
+  if (kFast) {
+    const float q0 = a * r;
+    const float q = std::fmaf(std::fmaf(-q0, s, a), r, q0);
+    return q0 < 1024.0f ? q : q0;
+  }
+  return a / s;
+#endif
+}
+
+// The window of given scales in which static_quotient<true> is exact.
+__host__ __device__ __forceinline__ bool static_scale_fast(float s) { return s >= 0x1p-92f && s <= 0x1p126f; }
 
 template <int FMT>
 __device__ __forceinline__ uint2 quant8(const uint4& v, const GroupScale& g) {
@@ -191,10 +235,13 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
 // ---------------------------------------------------------------------------
 // Activation quantization in the masked expert layout: expert e's tokens are
 // rows [e * cap, e * cap + counts[e]) of X; only those rows are quantized
-// (the padding rows' codes and scales are left as they are, and the masked
-// GEMM never reads them).  blockIdx.y = expert; the blocks of an expert
-// stride over its count * K/128 groups, 8 lanes per group as above.  A
-// count outside [0, cap] is clamped to it here; the masked GEMM reports it.
+// (the padding rows' codes and scales are left as they are: the masked GEMM
+// loads whole 128-row tiles, padding rows included, but every output row
+// depends on its own input row only and rows past the count are never
+// stored).  blockIdx.y = expert; the blocks of an expert stride over its
+// count * K/128 groups, 8 lanes per group as above.  A count outside
+// [0, cap] is clamped to it here and recorded in the status word
+// (kDevBadGroupOffsets), as the masked GEMM does.
 // ---------------------------------------------------------------------------
 template <int FMT>
 __global__ void __launch_bounds__(256) quant_act_masked_kernel(const uint16_t* __restrict__ X,
@@ -204,6 +251,8 @@ __global__ void __launch_bounds__(256) quant_act_masked_kernel(const uint16_t* _
   griddep_launch_dependents();
   const uint32_t e = blockIdx.y;
   const int32_t c = __ldg(counts + e);
+  if ((c < 0 || static_cast<uint32_t>(c) > cap) && blockIdx.x == 0 && threadIdx.x == 0)
+    record_status(kDevBadGroupOffsets);
   const uint32_t rows = c <= 0 ? 0u : (static_cast<uint32_t>(c) < cap ? static_cast<uint32_t>(c) : cap);
   const uint32_t total = rows * kb_div.d;
   const uint32_t lane = threadIdx.x & 31u;
@@ -400,22 +449,36 @@ __global__ void tensor_scale_finish_kernel(uint32_t* __restrict__ word) {
 
 // Static quantization with a given fp32 scale *scale (device):
 // code = E4M3(x / scale) over X [R, K], 16 bytes of input per thread step.
-__global__ void __launch_bounds__(256) quant_static_kernel(const uint16_t* __restrict__ X, uint32_t R, uint32_t K,
-                                                           uint64_t ldx, FastDiv chunk_div,
-                                                           const float* __restrict__ scale,
-                                                           uint8_t* __restrict__ Xq) {
-  griddep_launch_dependents();
-  GroupScale gs;
-  gs.s = __ldg(scale);
-  gs.r = __frcp_rn(gs.s);
-  gs.e8 = 0;
+// A scale that is not positive (<= 0 or NaN) is rejected: nothing is
+// written and the status word records kDevBadScale.  +inf is a valid scale
+// (every code becomes a signed zero).
+template <bool kFast>
+__device__ __forceinline__ void quant_static_run(const uint16_t* __restrict__ X, uint32_t R, uint64_t ldx, uint32_t K,
+                                                 const FastDiv& chunk_div, float s, uint8_t* __restrict__ Xq) {
+  const float r = kFast ? __frcp_rn(s) : 0.0f;
+  const auto div = [s, r](float x) { return static_quotient<kFast>(fabsf(x), s, r); };
   const uint32_t total = R * chunk_div.d;
   for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
     const uint32_t row = chunk_div.div(i);
     const uint32_t c = i - row * chunk_div.d;
     const uint4 v = ld_stream_v4(X + static_cast<uint64_t>(row) * ldx + c * 8u);
-    *reinterpret_cast<uint2*>(Xq + static_cast<uint64_t>(row) * K + c * 8u) = quant8<0>(v, gs);
+    *reinterpret_cast<uint2*>(Xq + static_cast<uint64_t>(row) * K + c * 8u) =
+        make_uint2(quant4_by(v.x, v.y, div), quant4_by(v.z, v.w, div));
   }
+}
+
+__global__ void __launch_bounds__(256) quant_static_kernel(const uint16_t* __restrict__ X, uint32_t R, uint32_t K,
+                                                           uint64_t ldx, FastDiv chunk_div,
+                                                           const float* __restrict__ scale,
+                                                           uint8_t* __restrict__ Xq) {
+  griddep_launch_dependents();
+  const float s = __ldg(scale);
+  if (!(s > 0.0f)) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) record_status(kDevBadScale);
+    return;
+  }
+  if (static_scale_fast(s)) quant_static_run<true>(X, R, ldx, K, chunk_div, s, Xq);
+  else quant_static_run<false>(X, R, ldx, K, chunk_div, s, Xq);
 }
 
 }  // namespace fgfp8

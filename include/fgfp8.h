@@ -162,12 +162,15 @@ fgfp8_status fgfp8_masked_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, 
  * The dynamic 1x128 activation quantizer of fgfp8_quant_act over the token
  * rows of the masked layout only: rows [e*cap, e*cap + counts[e]) of X for
  * every expert e.  Padding rows are not read, and their codes and scales
- * are left as they are (fgfp8_masked_gemm never reads them).
+ * are left as they are: fgfp8_masked_gemm loads them with their tile, but no
+ * output row depends on another row's input and rows past a count are never
+ * stored.
  *   X        DEVICE bf16 [E*cap, K], row stride ldx; Xq, Xs, ld_s as for
  *            fgfp8_quant_act with M = E*cap.
  *   counts   DEVICE int32 [E]; a count below 0 quantizes no row and one
- *            above cap quantizes cap rows (fgfp8_masked_gemm reports such
- *            a count).
+ *            above cap quantizes cap rows; either is recorded in the device
+ *            status word (fgfp8_check_device_status then returns
+ *            FGFP8_ERR_DEVICE), as fgfp8_masked_gemm does.
  * cap % 128 == 0, 1 <= E <= 65535; the other checks are those of
  * fgfp8_quant_act.  No counterpart on the pages: the decode step would
  * otherwise quantize every padding row.
@@ -240,6 +243,11 @@ fgfp8_status fgfp8_tensor_scale(const void* X, int64_t R, int64_t K, int64_t ldx
  * Static quantization with a given scale: Xq = E4M3(X / *scale), where
  * *scale is one float in device memory (a calibrated activation scale, or
  * the output of fgfp8_tensor_scale).  Layouts as for fgfp8_quant_rows.
+ * Any positive scale is accepted, subnormal and +inf included, and the codes
+ * equal those of the IEEE fp32 quotient x / scale for every finite bf16 x
+ * (a quotient beyond 448, or an infinite one, saturates to +-448).  A scale
+ * <= 0 or NaN is rejected on the device: no code is written and
+ * fgfp8_check_device_status returns FGFP8_ERR_DEVICE.
  */
 fgfp8_status fgfp8_quant_static(const void* X, int64_t R, int64_t K, int64_t ldx, const float* scale, uint8_t* Xq,
                                 void* stream);
@@ -341,7 +349,8 @@ fgfp8_status fgfp8_selftest_expired_wait(void* stream);
  * Synchronizes `stream`, then reads and clears the device status word that
  * the kernels set when they give up.  It returns FGFP8_OK,
  * FGFP8_ERR_TIMEOUT (a barrier wait ran past its one-second limit),
- * FGFP8_ERR_DEVICE (inconsistent group offsets) or FGFP8_ERR_CUDA.
+ * FGFP8_ERR_DEVICE (inconsistent group offsets, a masked count outside
+ * [0, cap], or a static scale that is not positive) or FGFP8_ERR_CUDA.
  */
 fgfp8_status fgfp8_check_device_status(void* stream);
 

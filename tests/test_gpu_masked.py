@@ -129,7 +129,8 @@ def test_quant_act_masked_token_rows_only(dev, fmt):
     """The masked quantizer writes exactly the token rows, bit-exact with the
     1x128 quantizer (and the oracle); padding rows (here NaN) are not read
     and their codes and scales stay as they were.  A count above cap
-    quantizes the whole block."""
+    quantizes the whole block, a negative one no row, and either is reported
+    through the device status word."""
     E, cap, K = 4, 128, 896
     counts = [5, 0, 128, 77]
     X = workloads.activations((E * cap, K), "normal_outliers", seed=31)
@@ -153,9 +154,20 @@ def test_quant_act_masked_token_rows_only(dev, fmt):
     Xq2 = torch.zeros_like(Xq_all)
     Xs2 = torch.zeros_like(Xs_all)
     fg.quant_act_masked(Xd, torch.tensor([0, cap + 9, 0, 0], dtype=torch.int32, device=dev), E, fmt, Xq=Xq2, Xs=Xs2)
-    fg.check_device_status()
+    with pytest.raises(fg.FGFP8Error) as ei:
+        fg.check_device_status()
+    assert ei.value.status == 7                                 # FGFP8_ERR_DEVICE
     blk = slice(cap, 2 * cap)
     assert torch.equal(Xq2[blk], Xq_all[blk])
+    # a negative count: no row of that expert, the others as usual, reported
+    Xq3 = torch.full((E * cap, K), 0xAB, dtype=torch.uint8, device=dev)
+    fg.quant_act_masked(Xd, torch.tensor([-3, 0, 0, 4], dtype=torch.int32, device=dev), E, fmt, Xq=Xq3, Xs=Xs2)
+    with pytest.raises(fg.FGFP8Error) as ei:
+        fg.check_device_status()
+    assert ei.value.status == 7
+    assert (Xq3[:cap] == 0xAB).all()
+    assert torch.equal(Xq3[3 * cap:3 * cap + 4], Xq_all[3 * cap:3 * cap + 4])
+    fg.check_device_status()                                    # cleared
 
 
 @pytest.mark.parametrize("fmt", [F32, UE8M0])

@@ -95,6 +95,64 @@ def test_tensor_scale_and_static_quant(dev, R, K):
         assert_codes_equal(to_np(Xq2), oracle.quant_static(bits16(X), given), f"static codes, scale {given}")
 
 
+def all_bf16_rows(K=128):
+    """Every finite bf16 value of both signs (65,280 of them, +-0 included),
+    as rows of K elements: the full range a static quotient x / s can meet."""
+    pos = np.arange(0, 0x7F80, dtype=np.uint16)
+    bits = np.concatenate([pos, pos | np.uint16(0x8000)])
+    rng = np.random.default_rng(11)
+    rng.shuffle(bits)
+    return torch.from_numpy(bits.view(np.int16).reshape(-1, K).copy()).view(torch.bfloat16)
+
+
+F32_MAX = float(np.finfo(np.float32).max)
+TINY_SUB = float(np.float32(2.0) ** -149)
+STATIC_EDGE_SCALES = [0.5, 1.0, 1e-39, 2.0 ** -126, 2.0 ** -127, 2.9387359e-39, TINY_SUB, 2.0 ** -92,
+                      float(np.nextafter(np.float32(2.0 ** -92), np.float32(0))), 2.0 ** 126,
+                      float(np.nextafter(np.float32(2.0 ** 126), np.float32(np.inf))), 2.0 ** 127, F32_MAX,
+                      float("inf"), 0.0031, 3.7e-12, 1.5e20]
+
+
+@pytest.mark.parametrize("scale", STATIC_EDGE_SCALES, ids=lambda v: f"{v:.6g}")
+def test_quant_static_every_bf16_value_at_edge_scales(dev, scale):
+    """A caller-given static scale meets every finite bf16 value: the codes
+    equal the oracle's E4M3(x / s) with the IEEE fp32 quotient bit for bit,
+    also where x / s overflows fp32 (|x| near the bf16 maximum over s = 0.5
+    saturates to 448, not NaN), for subnormal scales (1 / s overflows), at
+    the ends of the kernel's FMA window and for s = +inf."""
+    X = all_bf16_rows()
+    s = np.float32(scale)
+    Xq = fg.quant_static(X.to(dev), torch.tensor([s], dtype=torch.float32, device=dev))
+    fg.check_device_status()
+    assert_codes_equal(to_np(Xq), oracle.quant_static(bits16(X), s), f"static codes, scale {scale!r}")
+
+
+def test_quant_static_overflowing_quotient_saturates(dev):
+    """Rows holding +-3.0e38 and the bf16 maximum +-3.3895e38 over scale 0.5:
+    the quotient overflows fp32 and the code saturates to 0x7E / 0xFE."""
+    X = torch.zeros((2, 256), dtype=torch.bfloat16)
+    X[0, 0], X[0, 1], X[0, 2], X[0, 3] = 3.0e38, -3.0e38, 3.3895e38, -3.3895e38
+    X[1, 5], X[1, 6] = 1.0, -224.0
+    Xq = to_np(fg.quant_static(X.to(dev), torch.tensor([0.5], dtype=torch.float32, device=dev)))
+    fg.check_device_status()
+    assert list(Xq[0, :4]) == [0x7E, 0xFE, 0x7E, 0xFE]
+    assert_codes_equal(Xq, oracle.quant_static(bits16(X), np.float32(0.5)), "overflowing quotients")
+
+
+@pytest.mark.parametrize("bad", [0.0, -0.0, -1.0, float("nan"), -float("inf")])
+def test_quant_static_rejects_non_positive_scale(dev, bad):
+    """A scale <= 0 or NaN is reported through the device status word and
+    no code is written."""
+    X = workloads.activations((4, 256), "normal", seed=5).to(dev)
+    Xq = torch.full((4, 256), 0x5A, dtype=torch.uint8, device=dev)
+    fg.quant_static(X, torch.tensor([bad], dtype=torch.float32, device=dev), Xq=Xq)
+    with pytest.raises(fg.FGFP8Error) as e:
+        fg.check_device_status()
+    assert e.value.status == 7                     # FGFP8_ERR_DEVICE
+    assert bool((Xq == 0x5A).all())
+    fg.check_device_status()                      # the word was cleared
+
+
 def test_tensor_scale_zero_and_nan(dev):
     Z = torch.zeros((3, 256), dtype=torch.bfloat16, device=dev)
     assert float(fg.tensor_scale(Z)) == float(np.float32(1e-4) / np.float32(448.0))

@@ -1,7 +1,9 @@
 """Host-side checks of the quantizer's integer and floating-point arithmetic
-(CPU only): fast division by the number of K groups, and the FMA-based exact
+(CPU only): fast division by the number of K groups, the FMA-based exact
 quotient used instead of a per-element division (checked against IEEE
-division on every bf16 (element, amax) pair)."""
+division on every bf16 (element, amax) pair), and the static quantizer's
+quotient for caller-given scales (every bf16 magnitude against a sweep of
+scales from the smallest subnormal to +inf)."""
 import os
 import subprocess
 
@@ -22,3 +24,4 @@ def test_fastdiv_and_exact_quotient(tmp_path):
     print(r.stdout)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "quotient pairs:" in r.stdout and "mismatches: 0" in r.stdout
+    assert "static quotient pairs:" in r.stdout

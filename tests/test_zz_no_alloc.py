@@ -83,7 +83,10 @@ def test_noalloc_matches_linear_on_consecutive_calls():
         Xq_r, Xs_r = oracle.quant_act(bits16(X), fmt)
         Y_ref, S = oracle.gemm(Xq_r, Xs_r, Wq_r, Ws_r, fmt)
         what = f"call {i}: noalloc {M}x{N}x{K} fmt {fmt}"
-        # against the existing entry point, with the GEMM tolerance around its output
+        # against the existing entry point: the same kernels on the same inputs
+        # (only the scale rows' stride differs), so the same bits, which also
+        # lies within the GEMM tolerance around its output
+        assert torch.equal(outs[i], Y_lin), what + " differs from fgfp8_linear"
         assert_gemm_close(y_to_f64(outs[i]), y_to_f64(Y_lin), S, what + " vs fgfp8_linear")
         # and against the oracle
         assert_gemm_close(y_to_f64(outs[i]), Y_ref, S, what + " vs oracle")
