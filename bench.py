@@ -10,12 +10,18 @@ between them) for the per-kernel roofline.  Weights are quantized once before
 timing (fgfp8_quant_weight, reported separately), as a deployed layer holds
 pre-quantized weights.
 
-Default workload: the Llama-3-8B attention projection in prefill,
-X [4096, 4096] x W [4096, 4096], fp32 block scales.  Other workloads can be
-chosen with --workload (see workloads/), among them the same dense shapes
-with per-token x per-channel scales (the FP8_DYNAMIC scheme) or a static
-per-tensor activation scale, whose step is the row / tensor quantizer and
-the row/column-scaled GEMM.
+Default workload: the Llama-3-8B MLP in prefill as two W8A8 linear layers,
+the fused gate/up projection X [8192, 4096] x W [28672, 4096] (activations
+N(0, 1) with outliers) and then the down projection X [8192, 14336] x
+W [4096, 14336] (a post-SiLU-like heavy-tailed input), fp32 block scales,
+both bf16 outputs written: one step is two fgfp8_linear calls.  The roofline
+is taken on the gate/up GEMM (the dominant kernel) and the act-quant line on
+the 8192 x 14336 down-projection input (the largest activation).  Other
+workloads can be chosen with --workload (see workloads/), among them the
+attention projection 4096^3, the same dense shapes with per-token x
+per-channel scales (the FP8_DYNAMIC scheme) or a static per-tensor activation
+scale, whose step is the row / tensor quantizer and the row/column-scaled
+GEMM.
 
 Timing: W warm-up steps, then K timed steps.  L2 is flushed (a 256 MB write followed
 by a 256 MB read, so no dirty line is written back inside the next step)
@@ -70,6 +76,7 @@ WORKLOAD_ALIASES = {
     "llama_gate_up_dynamic": f"{workloads.LLAMA_GATE_UP.name}_fp8_dynamic",
     "llama_down_dynamic": f"{workloads.LLAMA_DOWN.name}_fp8_dynamic",
     "llama_mlp_fused": "llama3_8b_mlp_8192x4096x14336_swiglu_fused",
+    "llama_mlp_prefill": "llama3_8b_mlp_prefill_gate_up_8192x28672x4096_down_8192x4096x14336",
     "moe_decode_masked": workloads.MOE_DECODE.name,
     "moe_decode_masked_small": workloads.MOE_DECODE_SMALL.name,
     **{f"{a}_ue8m0": workloads.LLAMA_UE8M0[c.name].name
@@ -77,6 +84,8 @@ WORKLOAD_ALIASES = {
                     ("llama_down", workloads.LLAMA_DOWN))},
 }
 MLP_NAME = "llama3_8b_mlp_8192x4096x14336_swiglu_fused"
+PREFILL_NAME = "llama3_8b_mlp_prefill_gate_up_8192x28672x4096_down_8192x4096x14336"
+DEFAULT_WORKLOAD = "llama_mlp_prefill"
 
 
 def measured_peaks():
@@ -245,7 +254,7 @@ class DenseLayer:
                 "scales": "fp32" if c.fmt == 0 else "ue8m0", "x": c.x_kind}
 
     def host_io(self):
-        return self.X, self.Y
+        return [self.X], [self.Y]
 
     def gemm_kernel_name(self):
         if self.cfg.M <= 64:
@@ -316,10 +325,75 @@ class RowColLayer:
                 "scales": f"fp32, activations {x}, weights per output channel", "x": c.x_kind}
 
     def host_io(self):
-        return self.X, self.Y
+        return [self.X], [self.Y]
 
     def gemm_kernel_name(self):
         return "gemm_rowcol_kernel"
+
+
+class PrefillMLP:
+    """The Llama-3-8B MLP in prefill as two dense W8A8 linear layers, each one
+    fgfp8_linear call (the 1x128 quantizer, then the block-scaled GEMM as its
+    programmatic dependent), fp32 block scales: the fused gate/up projection
+    X [8192, 4096] (N(0, 1) with 0.1% outliers x50) x W [28672, 4096], then
+    the down projection X [8192, 14336] (sign(z)|z|^1.5, a post-SiLU-like
+    heavy tail) x W [4096, 14336].  Both bf16 outputs are written.  The down
+    input is its own seeded synthetic tensor, not derived from the gate/up
+    output (the SwiGLU chain between them is the separate fused workload)."""
+
+    launches_per_step = 4
+
+    def __init__(self, dev):
+        import fine_grained_fp8_token_b200 as fg
+        self.fg, self.dev = fg, dev
+        self.gu = DenseLayer(workloads.LLAMA_GATE_UP, dev)
+        self.down = DenseLayer(workloads.LLAMA_DOWN, dev)
+        self.X = self.gu.X
+
+    def quant_weight(self):
+        self.gu.quant_weight()
+
+    def linear(self, X=None):
+        self.gu.linear(None if X is None else X[0])
+        self.down.linear(None if X is None else X[1])
+
+    def kernel_steps(self):
+        """The step's kernels in launch order, for timing them apart."""
+        return [("quant_act_gate_up", self.gu.quant_act), ("gemm", self.gu.gemm),
+                ("quant_act", self.down.quant_act), ("gemm_down", self.down.gemm)]
+
+    def flops(self):
+        return self.gu.flops() + self.down.flops()
+
+    def kernel_flops(self):
+        return {"gemm": self.gu.flops(), "gemm_down": self.down.flops()}
+
+    def act_bytes(self):
+        return self.down.act_bytes()           # the act-quant line: the 8192 x 14336 input
+
+    def kernel_bytes(self):
+        return {"quant_act_gate_up": self.gu.act_bytes(), "quant_act": self.down.act_bytes(),
+                "gemm": self.gu.gemm_bytes(), "gemm_down": self.down.gemm_bytes()}
+
+    def gemm_bytes(self):
+        return self.gu.gemm_bytes()            # the roofline kernel: the gate/up GEMM
+
+    def weight_bytes(self):
+        return self.gu.weight_bytes()
+
+    def describe(self):
+        g, d = workloads.LLAMA_GATE_UP, workloads.LLAMA_DOWN
+        return {"workload": PREFILL_NAME,
+                "layers": [{"name": "gate_up", "M": g.M, "N": g.N, "K": g.K, "x": g.x_kind},
+                           {"name": "down", "M": d.M, "N": d.N, "K": d.K, "x": d.x_kind}],
+                "scales": "fp32 (1x128 activations, 128x128 weights)",
+                "roofline_kernel": "gate/up GEMM", "act_quant_line": "down-projection input 8192 x 14336"}
+
+    def host_io(self):
+        return [self.gu.X, self.down.X], [self.gu.Y, self.down.Y]
+
+    def gemm_kernel_name(self):
+        return "gemm_blockscaled_kernel (gate/up 8192x28672x4096)"
 
 
 class MLPLayer:
@@ -394,7 +468,7 @@ class MLPLayer:
                 "chain": "quant_act -> gate/up GEMM + SiLU*up + quant (fused) -> down GEMM"}
 
     def host_io(self):
-        return self.X, self.Y
+        return [self.X], [self.Y]
 
     def gemm_kernel_name(self):
         return "gemm_blockscaled_kernel (fused SwiGLU) + gemm_blockscaled_kernel"
@@ -474,7 +548,7 @@ class MaskedMoELayer:
                 "scales": "fp32" if c.fmt == 0 else "ue8m0"}
 
     def host_io(self):
-        return self.X, self.Y
+        return [self.X], [self.Y]
 
     def gemm_kernel_name(self):
         return ("gemm_blockscaled_kernel" if self.cfg.fmt == 0 else "gemm_mx_kernel") + " (masked)"
@@ -540,7 +614,7 @@ class MoELayer:
                 "max_rows_per_expert": int(self.r.counts.max()), "scales": "fp32" if c.fmt == 0 else "ue8m0"}
 
     def host_io(self):
-        return self.X, self.Y
+        return [self.X], [self.Y]
 
     def gemm_kernel_name(self):
         return ("gemm_blockscaled_kernel" if self.cfg.fmt == 0 else "gemm_mx_kernel") + " (grouped)"
@@ -553,6 +627,8 @@ def make_layer(name, dev, tokens=None):
             return MaskedMoELayer(cfg, dev)
     if name == MLP_NAME:
         return MLPLayer(dev, tokens)
+    if name == PREFILL_NAME:
+        return PrefillMLP(dev)
     if name in ROWCOL:
         cfg, scheme = ROWCOL[name]
         return RowColLayer(cfg, scheme, dev)
@@ -584,26 +660,28 @@ def whole_job_rate(world, units_per_rank, ms):
 def run_gpu(args, rank, world, dev):
     """Times the hot path on this rank.  The step is one call of the layer
     (fgfp8_linear / fgfp8_grouped_linear: the quantizer, then the GEMM as its
-    programmatic dependent), bracketed by CUDA events; a second pass of the
-    same length times the two kernels apart (an event between them) for the
-    per-kernel roofline."""
+    programmatic dependent; two such calls for the prefill MLP), bracketed by
+    CUDA events; a second pass of the same length times the kernels apart (an
+    event between consecutive ones) for the per-kernel roofline."""
     layer = make_layer(args.workload, dev, args.tokens)
     stream = torch.cuda.current_stream(dev)
     flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
     launches_per_step = getattr(layer, "launches_per_step", 2)
+    kernels = (layer.kernel_steps() if hasattr(layer, "kernel_steps")
+               else [("quant_act", layer.quant_act), ("gemm", layer.gemm)])
 
     for _ in range(args.warmup):
         flush_l2(flush_w, flush_r)
         layer.linear()
         flush_l2(flush_w, flush_r)
-        layer.quant_act()
-        layer.gemm()
+        for _, f in kernels:
+            f()
     layer.fg.check_device_status()
 
     n = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
-    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(kernels) + 1)] for _ in range(n)]
     sampler = ClockSampler(dev.index)
     if world > 1:
         torch.distributed.barrier()
@@ -622,18 +700,16 @@ def run_gpu(args, rank, world, dev):
     step_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(n)]
     total_ms = sum(step_ms)
 
-    # the two kernels timed apart (same flush between steps)
+    # the kernels timed apart (same flush between steps)
     for i in range(n):
         flush_l2(flush_w, flush_r)
         kev[i][0].record(stream)
-        layer.quant_act()
-        kev[i][1].record(stream)
-        layer.gemm()
-        kev[i][2].record(stream)
+        for j, (_, f) in enumerate(kernels):
+            f()
+            kev[i][j + 1].record(stream)
     torch.cuda.synchronize(dev)
     layer.fg.check_device_status()
-    quant_ms = [kev[i][0].elapsed_time(kev[i][1]) for i in range(n)]
-    gemm_ms = [kev[i][1].elapsed_time(kev[i][2]) for i in range(n)]
+    kern_ms = [sum(kev[i][j].elapsed_time(kev[i][j + 1]) for i in range(n)) for j in range(len(kernels))]
 
     # weight quantization (offline step, reported, not part of the step)
     wq_ms = []
@@ -648,33 +724,36 @@ def run_gpu(args, rank, world, dev):
 
     # end to end through the public API with host buffers: pinned X in,
     # quantize + GEMM, pinned Y out, copies inside the timed events
-    X_dev, Y_dev = layer.host_io()
-    X_host = torch.empty(X_dev.shape, dtype=X_dev.dtype, pin_memory=True)
-    X_host.copy_(X_dev)
-    Y_host = torch.empty(Y_dev.shape, dtype=Y_dev.dtype, pin_memory=True)
-    X_stage = torch.empty_like(X_dev)
+    X_devs, Y_devs = layer.host_io()
+    X_hosts = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in X_devs]
+    for xh, xd in zip(X_hosts, X_devs):
+        xh.copy_(xd)
+    Y_hosts = [torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for y in Y_devs]
+    X_stages = [torch.empty_like(x) for x in X_devs]
     e2e_ms = []
     e2e_steps = max(3, min(n, 10))
     for i in range(e2e_steps + 2):
         flush_l2(flush_w, flush_r)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        X_stage.copy_(X_host, non_blocking=True)
-        layer.linear(X_stage)
-        Y_host.copy_(Y_dev, non_blocking=True)
+        for xs, xh in zip(X_stages, X_hosts):
+            xs.copy_(xh, non_blocking=True)
+        layer.linear(X_stages[0] if len(X_stages) == 1 else X_stages)
+        for yh, yd in zip(Y_hosts, Y_devs):
+            yh.copy_(yd, non_blocking=True)
         b.record(stream)
         torch.cuda.synchronize(dev)
         if i >= 2:
             e2e_ms.append(a.elapsed_time(b))
-    h2d = X_host.numel() * X_host.element_size()
-    d2h = Y_host.numel() * Y_host.element_size()
+    h2d = sum(x.numel() * x.element_size() for x in X_hosts)
+    d2h = sum(y.numel() * y.element_size() for y in Y_hosts)
 
-    total_ms, gemm_total, quant_total, e2e_mean, wq_mean = max_over_ranks(
-        [total_ms, sum(gemm_ms), sum(quant_ms), statistics.mean(e2e_ms), statistics.mean(wq_ms)],
-        world, dev)
-    return layer, {"total_ms": total_ms, "gemm_ms": gemm_total / n, "quant_ms": quant_total / n,
-                   "e2e_ms": e2e_mean, "wq_ms": wq_mean, "clocks": clocks, "h2d": h2d, "d2h": d2h,
-                   "launches": launches_per_step * n}
+    vals = max_over_ranks([total_ms, *kern_ms, statistics.mean(e2e_ms), statistics.mean(wq_ms)], world, dev)
+    total_ms, kern_tot, e2e_mean, wq_mean = vals[0], vals[1:1 + len(kernels)], vals[-2], vals[-1]
+    kernel_ms = {name: t / n for (name, _), t in zip(kernels, kern_tot)}
+    return layer, {"total_ms": total_ms, "kernel_ms": kernel_ms, "gemm_ms": kernel_ms["gemm"],
+                   "quant_ms": kernel_ms["quant_act"], "e2e_ms": e2e_mean, "wq_ms": wq_mean, "clocks": clocks,
+                   "h2d": h2d, "d2h": d2h, "launches": launches_per_step * n}
 
 
 # ---------------------------------------------------------------- CPU oracle timing
@@ -711,6 +790,19 @@ class OracleSample:
             self.desc = (f"first {self.rows} of {MLPLayer.M} tokens through gate/up, SiLU * up, the 1x128 "
                          f"quantizer and down")
             return
+        if name == PREFILL_NAME:
+            b = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+            self.scheme, self.fmt = "prefill", 0
+            self.layers = []
+            for cfg in (workloads.LLAMA_GATE_UP, workloads.LLAMA_DOWN):
+                X, W = workloads.linear_inputs(cfg)
+                Wq, Ws = oracle.quant_weight(b(W), 0)
+                self.layers.append((np.ascontiguousarray(b(X[:rows])), Wq, Ws))
+            self.rows = self.layers[0][0].shape[0]
+            self.N, self.K = workloads.LLAMA_DOWN.N, workloads.LLAMA_GATE_UP.K
+            self.desc = (f"first {self.rows} of 8192 tokens through the gate/up layer [28672, 4096] and the down "
+                         f"layer [4096, 14336]")
+            return
         if name in ROWCOL:
             cfg, self.scheme = ROWCOL[name]
             X, W = workloads.linear_inputs(cfg)
@@ -745,6 +837,11 @@ class OracleSample:
         self.rows = self.X.shape[0]
 
     def step(self):
+        if self.scheme == "prefill":
+            for X, Wq, Ws in self.layers:
+                Xq, Xs = self.oracle.quant_act(X, 0)
+                self.oracle.gemm(Xq, Xs, Wq, Ws, 0)
+            return
         if self.scheme == "mlp":
             Xq, Xs = self.oracle.quant_act(self.X, 0)
             g, _ = self.oracle.gemm(Xq, Xs, self.Wq_g, self.Ws_g, 0)
@@ -765,6 +862,9 @@ class OracleSample:
         self.oracle.gemm(Xq, Xs, self.Wq, self.Ws, self.fmt)
 
     def flops(self):
+        if self.scheme == "prefill":
+            g, d = workloads.LLAMA_GATE_UP, workloads.LLAMA_DOWN
+            return 2.0 * self.rows * (g.N * g.K + d.N * d.K)
         if self.scheme == "mlp":
             return 2.0 * self.rows * (2 * MLPLayer.I * MLPLayer.K + MLPLayer.N_DOWN * MLPLayer.I)
         return 2.0 * self.rows * self.N * self.K
@@ -838,7 +938,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="fgfp8", choices=["fgfp8", "reference"])
-    ap.add_argument("--workload", default="llama_attn",
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     help="one of: " + ", ".join(WORKLOAD_ALIASES))
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (quick runs)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -869,7 +969,8 @@ def main():
     flops = layer.flops()
     value = whole_job_rate(world, flops, step_ms)
     fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
-    gemm_tflops = flops / (r["gemm_ms"] / 1e3) / 1e12
+    gemm_flops = layer.kernel_flops()["gemm"] if hasattr(layer, "kernel_flops") else flops
+    gemm_tflops = gemm_flops / (r["gemm_ms"] / 1e3) / 1e12
     gemm_gbs = layer.gemm_bytes() / (r["gemm_ms"] / 1e3) / 1e9
     act_gbs = layer.act_bytes() / (r["quant_ms"] / 1e3) / 1e9
     wq_gbs = layer.weight_bytes() / (r["wq_ms"] / 1e3) / 1e9
@@ -898,9 +999,10 @@ def main():
                           "bytes": layer.act_bytes()},
             "quant_weight_offline": {"us": 1e3 * r["wq_ms"], "gbs": wq_gbs, "frac_hbm": wq_gbs / peaks["hbm_gbs"],
                                      "bytes": layer.weight_bytes()},
-            "apart_sum_us": 1e3 * (r["quant_ms"] + r["gemm_ms"]),
+            "apart_sum_us": 1e3 * sum(r["kernel_ms"].values()),
         },
         "step_call": ("fgfp8_quant_act + fgfp8_gemm_swiglu_quant + fgfp8_gemm" if isinstance(layer, MLPLayer) else
+                      "fgfp8_linear (gate/up) + fgfp8_linear (down)" if isinstance(layer, PrefillMLP) else
                       "fgfp8_masked_linear" if isinstance(layer, MaskedMoELayer) else
                       "fgfp8_grouped_linear" if isinstance(layer, MoELayer) else
                       ("fgfp8_quant_rows + fgfp8_gemm_rowcol" if getattr(layer, "scheme", None) == "fp8_dynamic"
@@ -912,6 +1014,18 @@ def main():
         "clocks": r["clocks"],
         "peaks": peaks,
     }
+    if hasattr(layer, "kernel_flops"):
+        kb = layer.kernel_bytes()
+        for name, f in layer.kernel_flops().items():
+            if name != "gemm":
+                t = r["kernel_ms"][name] / 1e3
+                line["kernels"][name] = {"us": 1e6 * t, "tflops": f / t / 1e12, "frac_fp8_peak": f / t / 1e12 / fp8_peak,
+                                         "gbs": kb[name] / t / 1e9, "frac_hbm": kb[name] / t / 1e9 / peaks["hbm_gbs"]}
+        for name, b in kb.items():
+            if name.startswith("quant_act") and name != "quant_act":
+                t = r["kernel_ms"][name] / 1e3
+                line["kernels"][name] = {"us": 1e6 * t, "gbs": b / t / 1e9, "frac_hbm": b / t / 1e9 / peaks["hbm_gbs"],
+                                         "bytes": b}
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank == 0:
