@@ -47,6 +47,7 @@ SIGNATURES = {
     "fgfp8_masked_linear": (_INT, [_P, _I64, _P, _P, _I64, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _INT, _P]),
     "fgfp8_check_device_status": (_INT, [_P]),
     "fgfp8_selftest_expired_wait": (_INT, [_P]),
+    "fgfp8_selftest_gemm_timeout": (_INT, [_P, _P, _I64, _P, _P, _P, _I64, _I64, _I64, _INT, _I64, _P]),
 }
 
 _lock = threading.Lock()
@@ -115,6 +116,7 @@ fgfp8_quant_act_masked = _raw("fgfp8_quant_act_masked")
 fgfp8_masked_linear = _raw("fgfp8_masked_linear")
 fgfp8_check_device_status = _raw("fgfp8_check_device_status")
 fgfp8_selftest_expired_wait = _raw("fgfp8_selftest_expired_wait")
+fgfp8_selftest_gemm_timeout = _raw("fgfp8_selftest_gemm_timeout")
 
 
 def fgfp8_last_error_string() -> str:
@@ -379,6 +381,21 @@ def selftest_expired_wait(stream=None) -> None:
     """Launch the bounded-wait self-test (a wait that nothing completes; it
     gives up after one second and records a timeout in the status word)."""
     _check(fgfp8_selftest_expired_wait(_stream(stream)), "fgfp8_selftest_expired_wait")
+
+
+def selftest_gemm_timeout(Xq, Xs, Wq, Ws, fmt: int, withhold_kb: int, Y=None, stream=None):
+    """Run the dense GEMM with work item 0's K block withhold_kb never
+    requested (the GEMM self-test of its bounded waits).  Returns Y; the
+    status word then holds a timeout."""
+    import torch
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=Xq.device)
+    _check(fgfp8_selftest_gemm_timeout(Xq.data_ptr(), Xs.data_ptr(), Xs.shape[1], Wq.data_ptr(), Ws.data_ptr(),
+                                       Y.data_ptr(), M, N, K, fmt, withhold_kb, _stream(stream)),
+           "fgfp8_selftest_gemm_timeout")
+    return Y
 
 
 def check_device_status(stream=None) -> None:

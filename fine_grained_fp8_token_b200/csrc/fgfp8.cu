@@ -10,6 +10,7 @@
 #include <cstdio>
 #include <mutex>
 #include <set>
+#include <unordered_map>
 #include <utility>
 #include <string>
 
@@ -79,10 +80,47 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+// Encoded tensor maps, keyed by everything the encoding depends on (device,
+// base address, shape, row stride, box height).  A map holds no reference to
+// the memory: a later buffer at the same address with the same shape gets
+// the same, still valid, map.  The cache is cleared when it reaches
+// kMapCacheMax entries, so a caller cycling through many buffers never makes
+// it grow without bound.
+struct MapKey {
+  int dev;
+  const void* base;
+  uint64_t rows, cols, ld;
+  uint32_t box_rows;
+  bool operator==(const MapKey& o) const {
+    return dev == o.dev && base == o.base && rows == o.rows && cols == o.cols && ld == o.ld && box_rows == o.box_rows;
+  }
+};
+struct MapKeyHash {
+  size_t operator()(const MapKey& k) const {
+    uint64_t h = reinterpret_cast<uintptr_t>(k.base) * 0x9E3779B97F4A7C15ull;
+    for (uint64_t v : {static_cast<uint64_t>(k.dev), k.rows, k.cols, k.ld, static_cast<uint64_t>(k.box_rows)})
+      h = (h ^ v) * 0x100000001B3ull;
+    return static_cast<size_t>(h ^ (h >> 29));
+  }
+};
+constexpr size_t kMapCacheMax = 4096;
+
 // 2-D map over a row-major u8 matrix [rows, cols] (row stride ld bytes) with a
-// box of 128 columns (one 128-byte swizzle row) by box_rows rows.
+// box of 128 columns (one 128-byte swizzle row) by box_rows rows, on device
+// dev; encoded once per distinct key and then served from the cache.
 fgfp8_status make_map_u8_sw128(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
-                               uint32_t box_rows) {
+                               uint32_t box_rows, int dev) {
+  static std::mutex mu;
+  static std::unordered_map<MapKey, CUtensorMap, MapKeyHash> cache;
+  const MapKey key{dev, base, rows, cols, ld, box_rows};
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+      *map = it->second;
+      return FGFP8_OK;
+    }
+  }
   auto fn = encode_fn();
   if (!fn) return fail(FGFP8_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
   cuuint64_t dims[2] = {cols, rows};
@@ -93,6 +131,9 @@ fgfp8_status make_map_u8_sw128(CUtensorMap* map, const void* base, uint64_t rows
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(FGFP8_ERR_CUDA, "cuTensorMapEncodeTiled failed with code " + std::to_string(r));
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache.size() >= kMapCacheMax) cache.clear();
+  cache.emplace(key, *map);
   return FGFP8_OK;
 }
 
@@ -160,18 +201,18 @@ template <int BN, int CW, int FMT, bool kGrouped, bool kFuse = false>
 fgfp8_status launch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
                          void* Y, int64_t M, int64_t N, int64_t K, const int32_t* offs, int E, int64_t b_rows,
                          cudaStream_t stream, int dev, int sm_count, int early, int cap = 0, uint8_t* Hq = nullptr,
-                         float* Hs = nullptr, int64_t ld_h = 0) {
+                         float* Hs = nullptr, int64_t ld_h = 0, int withhold_kb = -1) {
   using C = fgfp8::GemmCfg<BN, CW>;
   CUtensorMap mA, mB, mBh;
   fgfp8_status st = make_map_u8_sw128(&mA, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
-                                      static_cast<uint64_t>(K), 128);
+                                      static_cast<uint64_t>(K), 128, dev);
   if (st != FGFP8_OK) return st;
   st = make_map_u8_sw128(&mB, Wq, static_cast<uint64_t>(b_rows), static_cast<uint64_t>(K), static_cast<uint64_t>(K),
-                         BN);
+                         BN, dev);
   if (st != FGFP8_OK) return st;
   // the same weights with a 128-row box, for half tiles
   st = make_map_u8_sw128(&mBh, Wq, static_cast<uint64_t>(b_rows), static_cast<uint64_t>(K), static_cast<uint64_t>(K),
-                         BN / 2);
+                         BN / 2, dev);
   if (st != FGFP8_OK) return st;
   auto kernel = fgfp8::gemm_blockscaled_kernel<BN, CW, FMT, kGrouped, kFuse>;
   st = set_smem(reinterpret_cast<const void*>(kernel), C::kSmemBytes, dev);
@@ -206,24 +247,24 @@ fgfp8_status launch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const 
                           mB, mBh, Xs, static_cast<uint32_t>(ld_s), Ws, reinterpret_cast<__nv_bfloat16*>(Y),
                           static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), offs, E, cap,
                           static_cast<int>(items), static_cast<int>(num_full), early, Hq, Hs,
-                          static_cast<uint32_t>(ld_h));
+                          static_cast<uint32_t>(ld_h), withhold_kb);
 }
 
 // UE8M0 launch with hardware block scaling (persistent, 128 x BN tiles).
 template <int BN, bool kGrouped>
 fgfp8_status launch_gemm_mx(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq, const void* Ws,
                             void* Y, int64_t M, int64_t N, int64_t K, const int32_t* offs, int E, int64_t b_rows,
-                            cudaStream_t stream, int dev, int sm_count, int early, int cap) {
+                            cudaStream_t stream, int dev, int sm_count, int early, int cap, int withhold_kb = -1) {
   using C = fgfp8::MxCfg<BN>;
   CUtensorMap mA, mB, mBh;
   fgfp8_status st = make_map_u8_sw128(&mA, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
-                                      static_cast<uint64_t>(K), 128);
+                                      static_cast<uint64_t>(K), 128, dev);
   if (st != FGFP8_OK) return st;
   st = make_map_u8_sw128(&mB, Wq, static_cast<uint64_t>(b_rows), static_cast<uint64_t>(K), static_cast<uint64_t>(K),
-                         C::kBN);
+                         C::kBN, dev);
   if (st != FGFP8_OK) return st;
   st = make_map_u8_sw128(&mBh, Wq, static_cast<uint64_t>(b_rows), static_cast<uint64_t>(K), static_cast<uint64_t>(K),
-                         C::kBN / 2);
+                         C::kBN / 2, dev);
   if (st != FGFP8_OK) return st;
   auto kernel = fgfp8::gemm_mx_kernel<BN, kGrouped>;
   st = set_smem(reinterpret_cast<const void*>(kernel), C::kSmemBytes, dev);
@@ -246,7 +287,7 @@ fgfp8_status launch_gemm_mx(const uint8_t* Xq, const void* Xs, int64_t ld_s, con
                           static_cast<uint32_t>(ld_s), reinterpret_cast<const uint8_t*>(Ws),
                           reinterpret_cast<__nv_bfloat16*>(Y), static_cast<int>(M), static_cast<int>(N),
                           static_cast<int>(K), offs, E, cap, static_cast<int>(items), static_cast<int>(num_full),
-                          early);
+                          early, withhold_kb);
 }
 
 template <bool kGrouped>
@@ -277,9 +318,9 @@ fgfp8_status launch_decode(const uint8_t* Xq, const void* Xs, int64_t ld_s, cons
   using C = fgfp8::DecodeCfg<BNT>;
   CUtensorMap mX, mW;
   fgfp8_status st = make_map_u8_sw128(&mX, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
-                                      static_cast<uint64_t>(K), BNT);
+                                      static_cast<uint64_t>(K), BNT, dev);
   if (st != FGFP8_OK) return st;
-  st = make_map_u8_sw128(&mW, Wq, static_cast<uint64_t>(N), static_cast<uint64_t>(K), static_cast<uint64_t>(K), 128);
+  st = make_map_u8_sw128(&mW, Wq, static_cast<uint64_t>(N), static_cast<uint64_t>(K), static_cast<uint64_t>(K), 128, dev);
   if (st != FGFP8_OK) return st;
   auto kernel = fgfp8::gemm_decode_kernel<BNT, FMT>;
   st = set_smem(reinterpret_cast<const void*>(kernel), C::kSmemBytes, dev);
@@ -297,9 +338,9 @@ fgfp8_status launch_decode_mx(const uint8_t* Xq, const void* Xs, int64_t ld_s, c
   using C = fgfp8::DecodeMxCfg<BNT>;
   CUtensorMap mX, mW;
   fgfp8_status st = make_map_u8_sw128(&mX, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
-                                      static_cast<uint64_t>(K), BNT);
+                                      static_cast<uint64_t>(K), BNT, dev);
   if (st != FGFP8_OK) return st;
-  st = make_map_u8_sw128(&mW, Wq, static_cast<uint64_t>(N), static_cast<uint64_t>(K), static_cast<uint64_t>(K), 128);
+  st = make_map_u8_sw128(&mW, Wq, static_cast<uint64_t>(N), static_cast<uint64_t>(K), static_cast<uint64_t>(K), 128, dev);
   if (st != FGFP8_OK) return st;
   auto kernel = fgfp8::gemm_decode_mx_kernel<BNT>;
   st = set_smem(reinterpret_cast<const void*>(kernel), C::kSmemBytes, dev);
@@ -333,12 +374,12 @@ fgfp8_status launch_gemm_rowcol(const uint8_t* Xq, const float* sx, int x_per_te
   using C = fgfp8::RowColCfg<BN>;
   CUtensorMap mA, mB, mBh;
   fgfp8_status st = make_map_u8_sw128(&mA, Xq, static_cast<uint64_t>(M), static_cast<uint64_t>(K),
-                                      static_cast<uint64_t>(K), 128);
+                                      static_cast<uint64_t>(K), 128, dev);
   if (st != FGFP8_OK) return st;
-  st = make_map_u8_sw128(&mB, Wq, static_cast<uint64_t>(N), static_cast<uint64_t>(K), static_cast<uint64_t>(K), BN);
+  st = make_map_u8_sw128(&mB, Wq, static_cast<uint64_t>(N), static_cast<uint64_t>(K), static_cast<uint64_t>(K), BN, dev);
   if (st != FGFP8_OK) return st;
   st = make_map_u8_sw128(&mBh, Wq, static_cast<uint64_t>(N), static_cast<uint64_t>(K), static_cast<uint64_t>(K),
-                         BN / 2);
+                         BN / 2, dev);
   if (st != FGFP8_OK) return st;
   auto kernel = fgfp8::gemm_rowcol_kernel<BN>;
   st = set_smem(reinterpret_cast<const void*>(kernel), C::kSmemBytes, dev);
@@ -853,6 +894,26 @@ fgfp8_status fgfp8_selftest_expired_wait(void* stream) {
   return check_launch("self-test launch");
 }
 
+fgfp8_status fgfp8_selftest_gemm_timeout(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq,
+                                         const void* Ws, void* Y, int64_t M, int64_t N, int64_t K, int fmt,
+                                         int64_t withhold_kb, void* stream) {
+  fgfp8_status st = check_gemm_common(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, fmt);
+  if (st != FGFP8_OK) return st;
+  if (M <= 64 || N % 256 != 0)
+    return fail(FGFP8_ERR_SHAPE, "the self-test runs the persistent 128x256-tile GEMM: M > 64 and N % 256 == 0");
+  if (withhold_kb < 0 || withhold_kb >= K / 128) return fail(FGFP8_ERR_INVALID_ARG, "withhold_kb must be in [0, K/128)");
+  int dev;
+  DeviceInfo info;
+  st = current_device(&dev, &info);
+  if (st != FGFP8_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int kb = static_cast<int>(withhold_kb);
+  if (fmt == FGFP8_SCALE_UE8M0)
+    return launch_gemm_mx<256, false>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, nullptr, 1, N, s, dev, info.sm_count, 0, 0, kb);
+  return launch_gemm<256, 128, 0, false>(Xq, Xs, ld_s, Wq, Ws, Y, M, N, K, nullptr, 1, N, s, dev, info.sm_count, 0, 0,
+                                         nullptr, nullptr, 0, kb);
+}
+
 fgfp8_status fgfp8_check_device_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
@@ -876,6 +937,8 @@ fgfp8_status fgfp8_check_device_status(void* stream) {
       return fail(FGFP8_ERR_DEVICE,
                   "group_offs is inconsistent (not a non-decreasing 0..M_total cover) or a masked count is outside "
                   "[0, cap]");
+    case fgfp8::kDevBadIndex:
+      return fail(FGFP8_ERR_DEVICE, "a debug-build index check failed (a tile, row, column or expert out of bounds)");
     case fgfp8::kDevBadScale:
       return fail(FGFP8_ERR_DEVICE, "the static quantizer's scale is not positive (<= 0 or NaN)");
     default:

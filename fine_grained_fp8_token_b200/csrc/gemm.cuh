@@ -247,7 +247,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
                             const __grid_constant__ CUtensorMap tmBh, const void* __restrict__ Xs, uint32_t ld_s,
                             const void* __restrict__ Ws, __nv_bfloat16* __restrict__ Y, int M, int N, int K,
                             const int32_t* __restrict__ group_offs, int E, int cap, int num_tiles, int num_full,
-                            int early_b, uint8_t* __restrict__ Hq, float* __restrict__ Hs, uint32_t ld_h) {
+                            int early_b, uint8_t* __restrict__ Hq, float* __restrict__ Hs, uint32_t ld_h,
+                            int withhold_kb) {
   using C = GemmCfg<BN, CW>;
   static_assert(!kFuse || (BN == 256 && CW == 128 && FMT == 0 && !kGrouped), "fused SwiGLU: dense fp32 256-wide");
   constexpr bool kHalfTiles = !kGrouped && BN == 256 && !kFuse;
@@ -299,6 +300,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
       m0 = (t / num_n) * C::kBM;
       expert = cap > 0 ? masked_expert(group_offs, E, cap, m0, row_end) : find_expert(group_offs, E, m0);
     }
+    FGFP8_DCHECK(t >= 0 && t < num_tiles && m0 >= 0 && m0 < M && n0 >= 0 && n0 + (half ? BN / 2 : BN) <= N &&
+                 expert >= -2 && expert < (kGrouped ? E : 1) && row_end <= M);
   };
 
   if (threadIdx.x == 0) {
@@ -374,6 +377,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
             ok = false;
             break;
           }
+          // fault injection (self-test only, withhold_kb < 0 in every product
+          // launch): work item 0 never requests K block withhold_kb, so the
+          // MMA's wait for it expires and every role unwinds
+          if (t == 0 && kb == withhold_kb) continue;
           if (it >= static_cast<uint32_t>(pre)) {
             mbar_arrive_expect_tx(&full[s], stage_tx);
             tma_load_2d(sB + s * C::kBBytes, mapB, &full[s], kb * C::kBK, b_row);
@@ -531,6 +538,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
         if (m < M) {
           const GroupScale gs = make_scale<0>(amax);
           const int i0 = n0 / 2;
+          FGFP8_DCHECK(i0 + 128 <= N / 2 && m < M);
           uint8_t* dst = Hq + static_cast<uint64_t>(m) * (N / 2) + i0 + (kGate ? 0 : 64);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
@@ -657,7 +665,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
           const int r = 4 * i + (lane >> 3), c = lane & 7;
           const uint4 v = *reinterpret_cast<const uint4*>(slot + r * 128 + ((c ^ (r & 7)) << 4));
           const int mr = m0 + quad * 32 + r;
-          if (mr < row_end) *reinterpret_cast<uint4*>(Y + static_cast<uint64_t>(mr) * N + n0 + col0 + p * 64 + c * 8) = v;
+          if (mr < row_end) {
+            FGFP8_DCHECK(mr < M && n0 + col0 + p * 64 + c * 8 + 8 <= N);
+            *reinterpret_cast<uint4*>(Y + static_cast<uint64_t>(mr) * N + n0 + col0 + p * 64 + c * 8) = v;
+          }
         }
         __syncwarp();
       }
@@ -747,7 +758,7 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
                    const __grid_constant__ CUtensorMap tmBh, const uint8_t* __restrict__ Xs, uint32_t ld_s,
                    const uint8_t* __restrict__ Ws, __nv_bfloat16* __restrict__ Y, int M, int N, int K,
                    const int32_t* __restrict__ group_offs, int E, int cap, int num_tiles, int num_full,
-                   int early_b) {
+                   int early_b, int withhold_kb) {
   using C = MxCfg<BN>;
   constexpr bool kHalfTiles = !kGrouped && BN == 256;
   static_assert(C::kSfCol + C::kSfSlots * C::kSfColsPerSlot <= C::kTmemCols, "TMEM columns");
@@ -796,6 +807,9 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
       m0 = (t / num_n) * C::kBM;
       expert = cap > 0 ? masked_expert(group_offs, E, cap, m0, row_end) : find_expert(group_offs, E, m0);
     }
+    FGFP8_DCHECK(t >= 0 && t < num_tiles && m0 >= 0 && m0 < M && n0 >= 0 &&
+                 n0 + (half ? C::kBN / 2 : C::kBN) <= N && expert >= -2 && expert < (kGrouped ? E : 1) &&
+                 row_end <= M);
   };
 
   if (threadIdx.x == 0) {
@@ -870,6 +884,7 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
             ok = false;
             break;
           }
+          if (t == 0 && kb == withhold_kb) continue;     // fault injection, as in the fp32-scale kernel
           if (it >= static_cast<uint32_t>(pre)) {
             mbar_arrive_expect_tx(&full[s], stage_tx);
             tma_load_2d(sB + s * C::kBBytes, mapB, &full[s], kb * C::kBK, expert * N + n0);
@@ -1062,6 +1077,7 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
       const int m = m0 + row;
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(ab * C::kBN + col0);
+      FGFP8_DCHECK(m >= row_end || (m < M && n0 + col0 + 128 <= N));
       __nv_bfloat16* yrow = Y + static_cast<uint64_t>(m) * N + n0 + col0;
       // the whole 128-column slice into registers first, so the accumulator
       // is handed back to the MMA before the (slower) global stores
@@ -1164,6 +1180,7 @@ __global__ void __launch_bounds__(RowColCfg<BN>::kThreads, 1)
     }
     m0 = (f % num_m) * C::kBM;
     n0 = (f / num_m) * C::kBN + h * (C::kBN / 2);
+    FGFP8_DCHECK(t >= 0 && t < num_tiles && m0 >= 0 && m0 < M && n0 >= 0 && n0 + (half ? C::kBN / 2 : C::kBN) <= N);
   };
 
   if (threadIdx.x == 0) {
@@ -1301,6 +1318,7 @@ __global__ void __launch_bounds__(RowColCfg<BN>::kThreads, 1)
       if (m < M) {
         const float a = __ldg(sx + (x_per_tensor ? 0 : m));
         const float w0 = w_per_tensor ? __ldg(sw) : 0.0f;
+        FGFP8_DCHECK(n0 + col0 + 128 <= N);
         __nv_bfloat16* yrow = Y + static_cast<uint64_t>(m) * N + n0 + col0;
         const float4* swv = reinterpret_cast<const float4*>(sw + n0 + col0);
 #pragma unroll
@@ -1480,7 +1498,10 @@ __global__ void __launch_bounds__(DecodeCfg<BNT>::kThreads, 1)
     if (ok && n < N) {
 #pragma unroll
       for (int m = 0; m < BNT; ++m)
-        if (m < M) Y[static_cast<uint64_t>(m) * N + n] = __float2bfloat16_rn(acc[m]);
+        if (m < M) {
+          FGFP8_DCHECK(m < BNT);
+          Y[static_cast<uint64_t>(m) * N + n] = __float2bfloat16_rn(acc[m]);
+        }
     }
   }
 
@@ -1702,7 +1723,10 @@ __global__ void __launch_bounds__(DecodeMxCfg<BNT>::kThreads, 1)
       if (n < N) {
 #pragma unroll
         for (int m = 0; m < BNT; ++m)
-          if (m < M) Y[static_cast<uint64_t>(m) * N + n] = __float2bfloat16_rn(__uint_as_float(p[m]));
+          if (m < M) {
+            FGFP8_DCHECK(m < BNT);
+            Y[static_cast<uint64_t>(m) * N + n] = __float2bfloat16_rn(__uint_as_float(p[m]));
+          }
       }
     } else if (lane == 0) {
       record_status(kDevTimeoutEpilogue);

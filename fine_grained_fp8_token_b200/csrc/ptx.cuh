@@ -17,6 +17,7 @@ enum : int {
   kDevBadGroupOffsets = 4,
   kDevTimeoutSelftest = 5,
   kDevBadScale = 6,
+  kDevBadIndex = 7,
 };
 
 // The device status word: the first nonzero code a kernel records stays
@@ -24,6 +25,23 @@ enum : int {
 __device__ int g_device_status;
 
 __device__ __forceinline__ void record_status(int code) { atomicCAS(&g_device_status, 0, code); }
+
+// Index checks of debug builds (-DFGFP8_DEBUG_CHECKS): tile origins, rows,
+// columns and experts are checked against the problem's bounds where they
+// are formed and before the global stores they address; a violation
+// records kDevBadIndex (the access itself is left as it is, so a debug run
+// finds the first bad index without changing what the kernel does).  In
+// release builds the checks compile to nothing.
+#ifdef FGFP8_DEBUG_CHECKS
+#define FGFP8_DCHECK(cond)                                           \
+  do {                                                               \
+    if (!(cond)) ::fgfp8::record_status(::fgfp8::kDevBadIndex);      \
+  } while (0)
+#else
+#define FGFP8_DCHECK(cond) \
+  do {                     \
+  } while (0)
+#endif
 
 // Upper bound on any single barrier wait.  A healthy wait here lasts at most
 // microseconds; one second means a lost arrival, and the kernel gives up.

@@ -221,6 +221,7 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
         codes.y = quant4<FMT>(v[u][0].z, v[u][0].w, gs);
         codes.z = quant4<FMT>(v[u][1].x, v[u][1].y, gs);
         codes.w = quant4<FMT>(v[u][1].z, v[u][1].w, gs);
+        FGFP8_DCHECK(m[u] < M && g[u] < kb_div.d);
         *reinterpret_cast<uint4*>(Xq + static_cast<uint64_t>(m[u]) * K + g[u] * kGroup + sub * 16u) = codes;
         if (sub == 0) {
           const uint64_t si = static_cast<uint64_t>(g[u]) * ld_s + m[u];
@@ -274,6 +275,7 @@ __global__ void __launch_bounds__(256) quant_act_masked_kernel(const uint16_t* _
     codes.y = quant4<FMT>(v0.z, v0.w, gs);
     codes.z = quant4<FMT>(v1.x, v1.y, gs);
     codes.w = quant4<FMT>(v1.z, v1.w, gs);
+    FGFP8_DCHECK(r < cap && g < kb_div.d);
     *reinterpret_cast<uint4*>(Xq + static_cast<uint64_t>(m) * K + g * kGroup + sub * 16u) = codes;
     if (sub == 0) {
       const uint64_t si = static_cast<uint64_t>(g) * ld_s + m;

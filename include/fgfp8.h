@@ -346,6 +346,25 @@ fgfp8_status fgfp8_linear_noalloc(const void* X, int64_t ldx, const uint8_t* Wq,
 fgfp8_status fgfp8_selftest_expired_wait(void* stream);
 
 /*
+ * Diagnostic with no counterpart on the pages: a self-test of the GEMM's own
+ * unwinding.  Runs the persistent dense GEMM (fmt F32: the promotion kernel;
+ * UE8M0: the block-scaled kernel) on the given operands, exactly as
+ * fgfp8_gemm would, except that the CTA holding work item 0 never requests
+ * the operand tiles of K block withhold_kb.  The MMA issuer's wait for them
+ * expires after its one-second limit, and with it the waits of the producer,
+ * the scale stager and the epilogue: each role records a timeout, stops
+ * issuing, waits (bounded) for the copies and MMAs it already issued, and
+ * the CTA frees TMEM and exits within a few seconds.  The other CTAs finish
+ * their tiles.  fgfp8_check_device_status then returns FGFP8_ERR_TIMEOUT,
+ * the context stays usable, and Y's tile 0 is left unspecified.
+ * Arguments as for fgfp8_gemm, with M > 64, N % 256 == 0 and
+ * 0 <= withhold_kb < K/128.
+ */
+fgfp8_status fgfp8_selftest_gemm_timeout(const uint8_t* Xq, const void* Xs, int64_t ld_s, const uint8_t* Wq,
+                                         const void* Ws, void* Y, int64_t M, int64_t N, int64_t K, int fmt,
+                                         int64_t withhold_kb, void* stream);
+
+/*
  * Synchronizes `stream`, then reads and clears the device status word that
  * the kernels set when they give up.  It returns FGFP8_OK,
  * FGFP8_ERR_TIMEOUT (a barrier wait ran past its one-second limit),

@@ -58,3 +58,26 @@ def assert_gemm_close(Y_gpu: np.ndarray, Y_ref: np.ndarray, S: np.ndarray, what:
         raise AssertionError(f"{what}: {len(bad)} of {ok.size} outside |d| <= 2^-7|ref| + 1e-4 S; first at {i}: "
                              f"gpu={Y_gpu[i]!r} ref={Y_ref[i]!r} S={S[i]!r}")
     assert np.isfinite(Y_gpu).all()
+
+
+class Guarded:
+    """A device output buffer with canary bytes on both sides: a stand-in for
+    a memory checker that finds writes outside an output (a wrong tile
+    index, row limit or leading dimension).  The inner tensor starts at a
+    256-byte boundary, so every alignment rule of the library holds."""
+
+    PAD = 4096
+    CANARY = 0xA5
+
+    def __init__(self, shape, dtype, device, fill=None):
+        n = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+        self.raw = torch.full((self.PAD + n + self.PAD,), self.CANARY, dtype=torch.uint8, device=device)
+        self.t = self.raw[self.PAD:self.PAD + n].view(dtype).view(*shape)
+        if fill is not None:
+            self.t.fill_(fill)
+
+    def check(self, what="output"):
+        lo = self.raw[:self.PAD]
+        hi = self.raw[-self.PAD:]
+        assert bool((lo == self.CANARY).all()), f"{what}: bytes written before the buffer"
+        assert bool((hi == self.CANARY).all()), f"{what}: bytes written after the buffer"

@@ -11,7 +11,7 @@ import torch
 import fine_grained_fp8_token_b200 as fg
 import oracle
 import workloads
-from parity import F32, UE8M0, assert_gemm_close, bits16, require_gpu, to_np, y_to_f64
+from parity import F32, UE8M0, Guarded, assert_gemm_close, bits16, require_gpu, to_np, y_to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -24,10 +24,20 @@ def dev():
 
 
 def gpu_linear(X_dev, W_dev, fmt):
-    Xq, Xs = fg.quant_act(X_dev, fmt)
+    """Quantizer, weight quantizer and GEMM, every output inside canary bytes."""
+    M, K = X_dev.shape
+    N = W_dev.shape[0]
+    sdt = torch.float32 if fmt == F32 else torch.uint8
+    gXq = Guarded((M, K), torch.uint8, X_dev.device)
+    gXs = Guarded((K // 128, fg.scale_rows(M, fmt)), sdt, X_dev.device, fill=0)
+    gY = Guarded((M, N), torch.bfloat16, X_dev.device)
+    Xq, Xs = fg.quant_act(X_dev, fmt, Xq=gXq.t, Xs=gXs.t)
     Wq, Ws = fg.quant_weight(W_dev, fmt)
-    Y = fg.gemm(Xq, Xs, Wq, Ws, fmt)
+    Y = fg.gemm(Xq, Xs, Wq, Ws, fmt, Y=gY.t)
     fg.check_device_status()
+    gXq.check("Xq")
+    gXs.check("Xs")
+    gY.check("Y")
     return Y
 
 
@@ -195,19 +205,28 @@ def test_grouped_gemm_empty_experts(dev):
     assert_gemm_close(y_to_f64(Y[torch.as_tensor(valid, device=dev)]), Y_ref, S, "grouped empty experts")
 
 
-def test_grouped_gemm_full_moe_sampled_rows(dev):
-    cfg = workloads.MOE
+@pytest.mark.parametrize("cfg", [workloads.MOE, workloads.MOE_F32], ids=lambda c: c.name)
+def test_grouped_gemm_full_moe_every_expert(dev, cfg):
+    """The full 256-expert layer the benchmark times (4096 tokens top-8,
+    Zipf-routed, 128-row padding), in both scale formats: the first and the
+    last token row of every expert segment, plus a middle row of the three
+    busiest experts, against the oracle with that expert's weights; every
+    padding row zero."""
     r, X, Y = build_moe(cfg, dev)
     starts = r.group_offs[:-1]
-    big = np.argsort(-r.counts)[:3]
-    pick = np.unique(np.r_[big, [cfg.E // 2, cfg.E - 1, 100]])
     rows = []
-    for e in pick:
+    for e in range(cfg.E):
         lo, n = int(starts[e]), int(r.counts[e])
-        rows += [lo, lo + n - 1, lo + n // 2]
+        if n:
+            rows += [lo, lo + n - 1]
+    for e in np.argsort(-r.counts)[:3]:
+        rows.append(int(starts[e]) + int(r.counts[e]) // 2)
     rows = np.unique(np.array(rows))
+    assert len(rows) >= 2 * int((r.counts > 0).sum())
     Y_ref, S = oracle_moe_rows(cfg, r, X, rows, dev)
     assert_gemm_close(y_to_f64(Y[torch.as_tensor(rows, device=dev)]), Y_ref, S, cfg.name)
+    pad = torch.as_tensor(np.where(r.row_token < 0)[0], device=dev)
+    assert (Y[pad].float() == 0).all()
 
 
 def test_grouped_gemm_bad_offsets_reported(dev):

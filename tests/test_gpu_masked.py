@@ -92,11 +92,12 @@ def test_masked_bad_count_reported(dev):
     fg.check_device_status()                                    # cleared
 
 
-def test_masked_full_decode_step_sampled_experts(dev):
+def test_masked_full_decode_step_every_expert(dev):
     """The 256-expert decode step the benchmark times (128 tokens top-8,
-    Zipf-routed, cap = 128, UE8M0): every token row of the busiest experts,
-    a middle one and the last active one against the oracle, every padding
-    row of every expert untouched."""
+    Zipf-routed, cap = 128, UE8M0): the first and last token row of every
+    active expert and every token row of the busiest experts, a middle one
+    and the last active one against the oracle; every padding row of every
+    expert untouched."""
     cfg, cap = workloads.MOE_DECODE, 128
     r = workloads.moe_routing(cfg)
     X = workloads.moe_masked_rows(workloads.moe_tokens(cfg, device=dev), r, cfg.E, cap)
@@ -110,14 +111,15 @@ def test_masked_full_decode_step_sampled_experts(dev):
     fg.masked_gemm(Xq, Xs, Wq, Ws, cnt, UE8M0, Y=Y)
     fg.check_device_status()
     active = np.where(r.counts > 0)[0]
-    pick = np.unique(np.r_[np.argsort(-r.counts)[:3], active[len(active) // 2], active[-1]])
-    for e in pick:
+    full = set(np.unique(np.r_[np.argsort(-r.counts)[:3], active[len(active) // 2], active[-1]]).tolist())
+    for e in active:
         c = int(r.counts[e])
-        rows = slice(int(e) * cap, int(e) * cap + c)
-        Xq_r, Xs_r = oracle.quant_act(bits16(X[rows]), UE8M0)
+        local = np.arange(c) if e in full else np.unique(np.r_[0, c - 1])
+        rows = int(e) * cap + local
+        Xq_r, Xs_r = oracle.quant_act(bits16(X[torch.as_tensor(rows, device=dev)]), UE8M0)
         Wq_r, Ws_r = oracle.quant_weight(bits16(workloads.moe_expert_weight(cfg, int(e), device=dev)), UE8M0)
         Y_ref, S = oracle.gemm(Xq_r, Xs_r, Wq_r, Ws_r, UE8M0)
-        assert_gemm_close(y_to_f64(Y[rows]), Y_ref, S, f"masked decode expert {e}")
+        assert_gemm_close(y_to_f64(Y[torch.as_tensor(rows, device=dev)]), Y_ref, S, f"masked decode expert {e}")
     pad = torch.ones(cfg.E * cap, dtype=torch.bool, device=dev)
     for e in active:
         pad[int(e) * cap:int(e) * cap + int(r.counts[e])] = False
