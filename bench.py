@@ -70,6 +70,7 @@ WORKLOAD_ALIASES = {
     "llama_attn": workloads.LLAMA_ATTN.name, "tiny": workloads.TINY.name,
     "llama_gate_up": workloads.LLAMA_GATE_UP.name, "llama_down": workloads.LLAMA_DOWN.name,
     **{f"ds_decode_m{m}": workloads.DS_DECODE[m].name for m in (1, 8, 32, 64)},
+    **{f"ds_decode_m{m}_layers": f"ds_decode_m{m}_layers" for m in (1, 8, 32, 64)},
     "moe": workloads.MOE.name, "moe_small": workloads.MOE_SMALL.name, "moe_fp32": workloads.MOE_F32.name,
     "llama_attn_dynamic": f"{workloads.LLAMA_ATTN.name}_fp8_dynamic",
     "llama_attn_static": f"{workloads.LLAMA_ATTN.name}_static_tensor",
@@ -262,6 +263,74 @@ class DenseLayer:
         return "gemm_blockscaled_kernel" if self.cfg.fmt == 0 else "gemm_mx_kernel"
 
 
+class DecodeSweep:
+    """Config-4 decode through L layers: M tokens (1..64) times L distinct
+    [18432, 7168] UE8M0 weights (8 x 132 MB, far above the 126 MB L2), as a
+    decode step walks through a model's layers.  One step is L calls of
+    fgfp8_linear (each quantizer, then its GEMM as the programmatic
+    dependent).  Timed apart, the L quantizers run back to back in one event
+    pair and the L GEMMs in another, so a kernel's time is its average over a
+    stream of launches rather than one launch behind an event (whose fixed
+    cost is several microseconds on this GPU)."""
+
+    LAYERS = 8
+
+    def __init__(self, cfg: workloads.Linear, dev):
+        import fine_grained_fp8_token_b200 as fg
+        self.fg, self.cfg, self.dev = fg, cfg, dev
+        self.layers = []
+        sdt = torch.float32 if cfg.fmt == 0 else torch.uint8
+        for i in range(self.LAYERS):
+            sub = workloads.replace(cfg, seed=cfg.seed + 16 * i)
+            d = DenseLayer(sub, dev)
+            del d.W                                       # keep only the quantized weight
+            self.layers.append(d)
+        self.W = workloads.weights((cfg.N, cfg.K), cfg.seed + 1, device=dev)   # for the weight-quantizer timing
+        self.Wq1 = torch.empty((cfg.N, cfg.K), dtype=torch.uint8, device=dev)
+        self.Ws1 = torch.empty((cfg.N // 128, cfg.K // 128), dtype=sdt, device=dev)
+        self.X = self.layers[0].X
+        self.launches_per_step = 2 * self.LAYERS
+
+    def quant_weight(self):
+        self.fg.quant_weight(self.W, self.cfg.fmt, Wq=self.Wq1, Ws=self.Ws1)
+
+    def quant_act(self, X=None):
+        for d in self.layers:
+            d.quant_act()
+
+    def gemm(self):
+        for d in self.layers:
+            d.gemm()
+
+    def linear(self, X=None):
+        for i, d in enumerate(self.layers):
+            d.linear(None if X is None else X[i])
+
+    def flops(self):
+        return self.LAYERS * self.layers[0].flops()
+
+    def act_bytes(self):
+        return self.LAYERS * self.layers[0].act_bytes()
+
+    def gemm_bytes(self):
+        return self.LAYERS * self.layers[0].gemm_bytes()
+
+    def weight_bytes(self):
+        return self.layers[0].weight_bytes()
+
+    def describe(self):
+        c = self.cfg
+        return {"workload": f"{c.name}_x{self.LAYERS}layers", "M": c.M, "N": c.N, "K": c.K, "layers": self.LAYERS,
+                "scales": "fp32" if c.fmt == 0 else "ue8m0", "x": c.x_kind,
+                "timing": "per-kernel times: L launches back to back in one event pair, divided by L"}
+
+    def host_io(self):
+        return [d.X for d in self.layers], [d.Y for d in self.layers]
+
+    def gemm_kernel_name(self):
+        return self.layers[0].gemm_kernel_name()
+
+
 class RowColLayer:
     """One dense layer with row / tensor scale granularity: per-output-channel
     weight scales (fgfp8_quant_rows on W) and either per-token activation
@@ -343,11 +412,16 @@ class PrefillMLP:
 
     launches_per_step = 4
 
-    def __init__(self, dev):
+    def __init__(self, dev, tokens=None):
         import fine_grained_fp8_token_b200 as fg
         self.fg, self.dev = fg, dev
-        self.gu = DenseLayer(workloads.LLAMA_GATE_UP, dev)
-        self.down = DenseLayer(workloads.LLAMA_DOWN, dev)
+        g, d = workloads.LLAMA_GATE_UP, workloads.LLAMA_DOWN
+        if tokens:                            # a smaller token batch (profiling captures)
+            g = workloads.replace(g, name=f"{g.name}@{tokens}tok", M=tokens)
+            d = workloads.replace(d, name=f"{d.name}@{tokens}tok", M=tokens)
+        self.tokens = tokens
+        self.gu = DenseLayer(g, dev)
+        self.down = DenseLayer(d, dev)
         self.X = self.gu.X
 
     def quant_weight(self):
@@ -382,8 +456,8 @@ class PrefillMLP:
         return self.gu.weight_bytes()
 
     def describe(self):
-        g, d = workloads.LLAMA_GATE_UP, workloads.LLAMA_DOWN
-        return {"workload": PREFILL_NAME,
+        g, d = self.gu.cfg, self.down.cfg
+        return {"workload": PREFILL_NAME if not self.tokens else f"{PREFILL_NAME}@{self.tokens}tok",
                 "layers": [{"name": "gate_up", "M": g.M, "N": g.N, "K": g.K, "x": g.x_kind},
                            {"name": "down", "M": d.M, "N": d.N, "K": d.K, "x": d.x_kind}],
                 "scales": "fp32 (1x128 activations, 128x128 weights)",
@@ -628,14 +702,20 @@ def make_layer(name, dev, tokens=None):
     if name == MLP_NAME:
         return MLPLayer(dev, tokens)
     if name == PREFILL_NAME:
-        return PrefillMLP(dev)
+        return PrefillMLP(dev, tokens)
     if name in ROWCOL:
         cfg, scheme = ROWCOL[name]
         return RowColLayer(cfg, scheme, dev)
     for cfg in (workloads.MOE, workloads.MOE_SMALL, workloads.MOE_F32):
         if name == cfg.name:
             return MoELayer(cfg, dev)
-    return DenseLayer(workloads.LINEARS[name], dev)
+    for m, cfg in workloads.DS_DECODE.items():
+        if name in (f"{cfg.name}_x{DecodeSweep.LAYERS}layers", f"ds_decode_m{m}_layers"):
+            return DecodeSweep(cfg, dev)
+    cfg = workloads.LINEARS[name]
+    if tokens:                                # a smaller token batch of the same layer (profiling captures)
+        cfg = workloads.replace(cfg, name=f"{cfg.name}@{tokens}tok", M=tokens)
+    return DenseLayer(cfg, dev)
 
 
 # ---------------------------------------------------------------- ranks
@@ -827,7 +907,10 @@ class OracleSample:
             self.N, self.K, self.fmt = cfg.N, cfg.K, cfg.fmt
             self.desc = f"{min(rows, len(tok))} routed rows of expert {e} x its [4096, 7168] weight"
         else:
-            cfg = workloads.LINEARS[name]
+            cfg = workloads.LINEARS.get(name)
+            if cfg is None:                             # the decode sweep: one layer's sample
+                cfg = next(c for m, c in workloads.DS_DECODE.items()
+                           if name in (f"{c.name}_x{DecodeSweep.LAYERS}layers", f"ds_decode_m{m}_layers"))
             X, W = workloads.linear_inputs(cfg)
             X = X[:rows]
             self.N, self.K, self.fmt = cfg.N, cfg.K, cfg.fmt
@@ -943,7 +1026,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (quick runs)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--tokens", type=int, default=None,
-                    help="token batch of the fused MLP workload (default: its 8192; smaller for profiling captures)")
+                    help="token batch M of the MLP and dense workloads (default: the workload's own; smaller for "
+                         "profiling captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

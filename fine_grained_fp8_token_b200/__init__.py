@@ -46,6 +46,7 @@ SIGNATURES = {
     "fgfp8_quant_act_masked": (_INT, [_P, _I64, _P, _I32, _I64, _I64, _P, _P, _I64, _INT, _P]),
     "fgfp8_masked_linear": (_INT, [_P, _I64, _P, _P, _I64, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _INT, _P]),
     "fgfp8_check_device_status": (_INT, [_P]),
+    "fgfp8_gather_cols": (_INT, [_P, _I64, _I64, _I64, _P, _P]),
     "fgfp8_selftest_expired_wait": (_INT, [_P]),
     "fgfp8_selftest_gemm_timeout": (_INT, [_P, _P, _I64, _P, _P, _P, _I64, _I64, _I64, _INT, _I64, _P]),
 }
@@ -115,6 +116,7 @@ fgfp8_masked_gemm = _raw("fgfp8_masked_gemm")
 fgfp8_quant_act_masked = _raw("fgfp8_quant_act_masked")
 fgfp8_masked_linear = _raw("fgfp8_masked_linear")
 fgfp8_check_device_status = _raw("fgfp8_check_device_status")
+fgfp8_gather_cols = _raw("fgfp8_gather_cols")
 fgfp8_selftest_expired_wait = _raw("fgfp8_selftest_expired_wait")
 fgfp8_selftest_gemm_timeout = _raw("fgfp8_selftest_gemm_timeout")
 
@@ -381,6 +383,17 @@ def selftest_expired_wait(stream=None) -> None:
     """Launch the bounded-wait self-test (a wait that nothing completes; it
     gives up after one second and records a timeout in the status word)."""
     _check(fgfp8_selftest_expired_wait(_stream(stream)), "fgfp8_selftest_expired_wait")
+
+
+def gather_cols(parts, Y=None, stream=None):
+    """parts bf16 [P, M, n] (an all-gather of per-rank column blocks) ->
+    Y bf16 [M, P * n] with Y[m, p * n + j] = parts[p, m, j]."""
+    import torch
+    P, M, n = parts.shape
+    if Y is None:
+        Y = torch.empty((M, P * n), dtype=parts.dtype, device=parts.device)
+    _check(fgfp8_gather_cols(parts.data_ptr(), P, M, n, Y.data_ptr(), _stream(stream)), "fgfp8_gather_cols")
+    return Y
 
 
 def selftest_gemm_timeout(Xq, Xs, Wq, Ws, fmt: int, withhold_kb: int, Y=None, stream=None):

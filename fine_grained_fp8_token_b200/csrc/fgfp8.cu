@@ -16,6 +16,7 @@
 
 #include "fgfp8.h"
 #include "gemm.cuh"
+#include "layout.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
 
@@ -883,6 +884,26 @@ fgfp8_status fgfp8_gemm_swiglu_quant(const uint8_t* Xq, const float* Xs, int64_t
   return launch_gemm<256, 128, 0, false, true>(Xq, Xs, ld_s, Wq_gu, Ws_gu, nullptr, M, 2 * I, K, nullptr, 1, 2 * I,
                                                reinterpret_cast<cudaStream_t>(stream), dev, info.sm_count, 0, 0, Hq,
                                                Hs, ld_h);
+}
+
+fgfp8_status fgfp8_gather_cols(const void* parts, int64_t P, int64_t M, int64_t n, void* Y, void* stream) {
+  if (P < 0 || M < 0 || n < 0) return fail(FGFP8_ERR_INVALID_ARG, "negative size");
+  if (P == 0 || M == 0 || n == 0) return ok();
+  if (n % 8 != 0) return fail(FGFP8_ERR_SHAPE, "n must be a multiple of 8 (16-byte rows)");
+  if (P * M * (n / 8) >= (int64_t(1) << 32) || M >= (int64_t(1) << 31))
+    return fail(FGFP8_ERR_SHAPE, "P * M * n / 8 must be < 2^32");
+  if (!parts || !Y) return fail(FGFP8_ERR_INVALID_ARG, "parts or Y is NULL");
+  if (!aligned(parts, 16) || !aligned(Y, 16)) return fail(FGFP8_ERR_ALIGN, "parts and Y must be 16-byte aligned");
+  int dev;
+  DeviceInfo info;
+  fgfp8_status st = current_device(&dev, &info);
+  if (st != FGFP8_OK) return st;
+  const uint32_t total = static_cast<uint32_t>(P * M * (n / 8));
+  fgfp8::gather_cols_kernel<<<grid_stride_blocks(total, info.sm_count), 256, 0,
+                              reinterpret_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint4*>(parts), total, fgfp8::FastDiv(static_cast<uint32_t>(n / 8)),
+      fgfp8::FastDiv(static_cast<uint32_t>(M)), reinterpret_cast<uint4*>(Y));
+  return check_launch("gather_cols launch");
 }
 
 fgfp8_status fgfp8_selftest_expired_wait(void* stream) {

@@ -299,6 +299,19 @@ fgfp8_status fgfp8_gemm_swiglu_quant(const uint8_t* Xq, const float* Xs, int64_t
                                      const float* Ws_gu, uint8_t* Hq, float* Hs, int64_t ld_h, int64_t M, int64_t I,
                                      int64_t K, void* stream);
 
+/*
+ * Output layout of a tensor-parallel column split (no counterpart on the
+ * pages, which run the layer on one GPU): when P ranks each hold n = N/P of
+ * the weight's output rows (whole 128-row blocks with their block scales)
+ * and compute their part of Y with fgfp8_linear / fgfp8_gemm, an all-gather
+ * stacks the parts as parts bf16 [P, M, n]; this call writes them as
+ * Y bf16 [M, P * n], Y[m, p * n + j] = parts[p, m, j].  Both buffers are in
+ * this device's memory (the all-gather brings remote parts in first).
+ *   parts, Y  16-byte aligned, contiguous; n % 8 == 0; P * M * n / 8 < 2^32.
+ * P, M or n == 0 is a no-op.
+ */
+fgfp8_status fgfp8_gather_cols(const void* parts, int64_t P, int64_t M, int64_t n, void* Y, void* stream);
+
 /* Size of the static scratch of fgfp8_linear_noalloc: 32 MiB per device. */
 #define FGFP8_NOALLOC_SCRATCH_BYTES (32u << 20)
 
