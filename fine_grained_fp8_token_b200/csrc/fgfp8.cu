@@ -195,6 +195,16 @@ fgfp8_status check_act_scales(const void* Xs, int64_t ld_s, int64_t M, int fmt) 
   return FGFP8_OK;
 }
 
+// M tiles per band of the dense tile order (see grouped_tile): the plain
+// M-fastest order while the activation codes fit comfortably in L2 (every
+// weight tile is then read once), else bands of 16 M tiles, whose activation
+// rows and the weight tiles a wave touches fit in L2 together.
+int dense_group_m(int64_t M, int64_t K, int bm) {
+  const int64_t num_m = (M + bm - 1) / bm;
+  if (M * K <= (int64_t(48) << 20)) return static_cast<int>(num_m);
+  return static_cast<int>(num_m < 16 ? num_m : 16);
+}
+
 // Launch one GEMM instantiation as a persistent grid (one CTA per SM at most).
 // kFuse: the SwiGLU gate/up projection writing the down projection's
 // quantized input (Hq, Hs, ld_h) instead of Y.
@@ -248,7 +258,7 @@ fgfp8_status launch_gemm(const uint8_t* Xq, const void* Xs, int64_t ld_s, const 
                           mB, mBh, Xs, static_cast<uint32_t>(ld_s), Ws, reinterpret_cast<__nv_bfloat16*>(Y),
                           static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), offs, E, cap,
                           static_cast<int>(items), static_cast<int>(num_full), early, Hq, Hs,
-                          static_cast<uint32_t>(ld_h), withhold_kb);
+                          static_cast<uint32_t>(ld_h), withhold_kb, dense_group_m(M, K, C::kBM));
 }
 
 // UE8M0 launch with hardware block scaling (persistent, 128 x BN tiles).
@@ -288,7 +298,7 @@ fgfp8_status launch_gemm_mx(const uint8_t* Xq, const void* Xs, int64_t ld_s, con
                           static_cast<uint32_t>(ld_s), reinterpret_cast<const uint8_t*>(Ws),
                           reinterpret_cast<__nv_bfloat16*>(Y), static_cast<int>(M), static_cast<int>(N),
                           static_cast<int>(K), offs, E, cap, static_cast<int>(items), static_cast<int>(num_full),
-                          early, withhold_kb);
+                          early, withhold_kb, dense_group_m(M, K, C::kBM));
 }
 
 template <bool kGrouped>
@@ -400,7 +410,8 @@ fgfp8_status launch_gemm_rowcol(const uint8_t* Xq, const float* sx, int x_per_te
   return launch_dependent(kernel, static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, stream,
                           "row/column-scaled gemm launch", mA, mB, mBh, sx, x_per_tensor, sw, w_per_tensor,
                           reinterpret_cast<__nv_bfloat16*>(Y), static_cast<int>(M), static_cast<int>(N),
-                          static_cast<int>(K), static_cast<int>(items), static_cast<int>(num_full));
+                          static_cast<int>(K), static_cast<int>(items), static_cast<int>(num_full),
+                          dense_group_m(M, K, C::kBM));
 }
 
 // Shared checks of the row / tensor quantizers' input X bf16 [R, K] (row

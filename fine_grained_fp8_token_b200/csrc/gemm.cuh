@@ -117,6 +117,21 @@ __device__ __forceinline__ float combine_raw(uint32_t a, uint32_t w) {
 // Depth (in K blocks) of the scale prefetch ring of the promotion warps.
 constexpr int kScaleAhead = 2;
 
+// Dense tile f -> (M tile, N tile) in bands of group_m M tiles: within a
+// band the M index runs fastest, then N; the bands follow each other.  A
+// wave then covers about group_m M tiles x (wave / group_m) N tiles, so the
+// activation and weight tiles it touches stay L2-resident together.  With
+// group_m >= num_m this is the plain M-fastest order (the whole activation
+// matrix resident while every weight tile is read once).
+__device__ __forceinline__ void grouped_tile(int f, int num_m, int num_n, int group_m, int& mi, int& ni) {
+  const int band_tiles = group_m * num_n;
+  const int band = f / band_tiles;
+  const int r = f - band * band_tiles;
+  const int rows = min(group_m, num_m - band * group_m);
+  mi = band * group_m + r % rows;
+  ni = r / rows;
+}
+
 // Expert owning row m: the e with offs[e] <= m < offs[e+1] (binary search),
 // or -1 when the offsets are inconsistent with m.
 __device__ __forceinline__ int find_expert(const int32_t* __restrict__ offs, int E, int m) {
@@ -248,7 +263,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
                             const void* __restrict__ Ws, __nv_bfloat16* __restrict__ Y, int M, int N, int K,
                             const int32_t* __restrict__ group_offs, int E, int cap, int num_tiles, int num_full,
                             int early_b, uint8_t* __restrict__ Hq, float* __restrict__ Hs, uint32_t ld_h,
-                            int withhold_kb) {
+                            int withhold_kb, int group_m) {
   using C = GemmCfg<BN, CW>;
   static_assert(!kFuse || (BN == 256 && CW == 128 && FMT == 0 && !kGrouped), "fused SwiGLU: dense fp32 256-wide");
   constexpr bool kHalfTiles = !kGrouped && BN == 256 && !kFuse;
@@ -292,8 +307,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
         h = (t - num_full) & 1;
         half = true;
       }
-      m0 = (f % num_m) * C::kBM;
-      n0 = (f / num_m) * BN + h * (BN / 2);
+      int mi, ni;
+      grouped_tile(f, num_m, num_n, group_m, mi, ni);
+      m0 = mi * C::kBM;
+      n0 = ni * BN + h * (BN / 2);
       expert = 0;
     } else {
       n0 = (t % num_n) * BN;
@@ -758,7 +775,7 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
                    const __grid_constant__ CUtensorMap tmBh, const uint8_t* __restrict__ Xs, uint32_t ld_s,
                    const uint8_t* __restrict__ Ws, __nv_bfloat16* __restrict__ Y, int M, int N, int K,
                    const int32_t* __restrict__ group_offs, int E, int cap, int num_tiles, int num_full,
-                   int early_b, int withhold_kb) {
+                   int early_b, int withhold_kb, int group_m) {
   using C = MxCfg<BN>;
   constexpr bool kHalfTiles = !kGrouped && BN == 256;
   static_assert(C::kSfCol + C::kSfSlots * C::kSfColsPerSlot <= C::kTmemCols, "TMEM columns");
@@ -799,8 +816,10 @@ __global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
         h = (t - num_full) & 1;
         half = true;
       }
-      m0 = (f % num_m) * C::kBM;
-      n0 = (f / num_m) * C::kBN + h * (C::kBN / 2);
+      int mi, ni;
+      grouped_tile(f, num_m, num_n, group_m, mi, ni);
+      m0 = mi * C::kBM;
+      n0 = ni * C::kBN + h * (C::kBN / 2);
       expert = 0;
     } else {
       n0 = (t % num_n) * C::kBN;
@@ -1150,7 +1169,7 @@ __global__ void __launch_bounds__(RowColCfg<BN>::kThreads, 1)
     gemm_rowcol_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const __grid_constant__ CUtensorMap tmBh, const float* __restrict__ sx, int x_per_tensor,
                        const float* __restrict__ sw, int w_per_tensor, __nv_bfloat16* __restrict__ Y, int M, int N,
-                       int K, int num_tiles, int num_full) {
+                       int K, int num_tiles, int num_full, int group_m) {
   using C = RowColCfg<BN>;
   constexpr bool kHalfTiles = BN == 256;
   extern __shared__ uint8_t smem_raw[];
@@ -1168,8 +1187,10 @@ __global__ void __launch_bounds__(RowColCfg<BN>::kThreads, 1)
   const int lane = threadIdx.x & 31;
   const int KB = K / C::kBK;
   const int num_m = (M + C::kBM - 1) / C::kBM;
-  // work item t -> (m0, n0, half), M-fastest; items t >= num_full are the
-  // 128 x 128 halves of the remaining full tiles (as in the fp32-scale kernel)
+  const int num_n = N / C::kBN;
+  // work item t -> (m0, n0, half) in the banded order of grouped_tile; items
+  // t >= num_full are the 128 x 128 halves of the remaining full tiles (as in
+  // the fp32-scale kernel)
   auto coords = [&](int t, int& m0, int& n0, bool& half) {
     int f = t, h = 0;
     half = false;
@@ -1178,8 +1199,10 @@ __global__ void __launch_bounds__(RowColCfg<BN>::kThreads, 1)
       h = (t - num_full) & 1;
       half = true;
     }
-    m0 = (f % num_m) * C::kBM;
-    n0 = (f / num_m) * C::kBN + h * (C::kBN / 2);
+    int mi, ni;
+    grouped_tile(f, num_m, num_n, group_m, mi, ni);
+    m0 = mi * C::kBM;
+    n0 = ni * C::kBN + h * (C::kBN / 2);
     FGFP8_DCHECK(t >= 0 && t < num_tiles && m0 >= 0 && m0 < M && n0 >= 0 && n0 + (half ? C::kBN / 2 : C::kBN) <= N);
   };
 
