@@ -736,6 +736,62 @@ def whole_job_rate(world, units_per_rank, ms):
     return world * units_per_rank / (ms / 1e3) / 1e12
 
 
+# ---------------------------------------------------------------- end to end
+E2E_CHUNKS = 4
+
+
+def streamed_parts(layer):
+    """The dense layers of a step whose token rows can be streamed through
+    host copies in chunks (each output row depends on its own input row
+    only), or None for workloads run in one piece."""
+    if isinstance(layer, PrefillMLP):
+        return [layer.gu, layer.down]
+    if type(layer) is DenseLayer and layer.cfg.M >= 1024:
+        return [layer]
+    return None
+
+
+def e2e_streamed(parts, X_hosts, X_stages, Y_hosts, stream, dev, start):
+    """One end-to-end step of the dense layers `parts`, streamed over
+    E2E_CHUNKS token chunks each: chunk copies host -> device on one stream,
+    fgfp8_linear of the chunk on the compute stream once its rows are in,
+    and the chunk's output device -> host on a third stream once computed,
+    so the two copy directions overlap each other and the compute.  Every
+    stream starts after `start` and the compute stream waits for the last
+    copy out, so an event recorded next on it closes the step."""
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    s_in.wait_event(start)
+    s_out.wait_event(start)
+    chunks = []                                  # (part index, r0, r1)
+    for i, d in enumerate(parts):
+        M = d.cfg.M
+        bounds = [(M * c // E2E_CHUNKS) // 16 * 16 for c in range(E2E_CHUNKS)] + [M]
+        chunks += [(i, r0, r1) for r0, r1 in zip(bounds, bounds[1:]) if r1 > r0]
+    ev_in = []
+    for i, r0, r1 in chunks:
+        with torch.cuda.stream(s_in):
+            X_stages[i][r0:r1].copy_(X_hosts[i][r0:r1], non_blocking=True)
+        e = torch.cuda.Event()
+        e.record(s_in)
+        ev_in.append(e)
+    ev_c = []
+    for (i, r0, r1), e in zip(chunks, ev_in):
+        d = parts[i]
+        stream.wait_event(e)
+        d.fg.linear(X_stages[i][r0:r1], d.Wq, d.Ws, d.cfg.fmt, Y=d.Y[r0:r1], Xq=d.Xq[r0:r1], Xs=d.Xs[:, r0:],
+                    ld_s=d.ld_s, stream=stream)
+        e2 = torch.cuda.Event()
+        e2.record(stream)
+        ev_c.append(e2)
+    for (i, r0, r1), e2 in zip(chunks, ev_c):
+        s_out.wait_event(e2)
+        with torch.cuda.stream(s_out):
+            Y_hosts[i][r0:r1].copy_(parts[i].Y[r0:r1], non_blocking=True)
+    done = torch.cuda.Event()
+    done.record(s_out)
+    stream.wait_event(done)
+
+
 # ---------------------------------------------------------------- timing
 def run_gpu(args, rank, world, dev):
     """Times the hot path on this rank.  The step is one call of the layer
@@ -812,15 +868,19 @@ def run_gpu(args, rank, world, dev):
     X_stages = [torch.empty_like(x) for x in X_devs]
     e2e_ms = []
     e2e_steps = max(3, min(n, 10))
+    parts = streamed_parts(layer)
     for i in range(e2e_steps + 2):
         flush_l2(flush_w, flush_r)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        for xs, xh in zip(X_stages, X_hosts):
-            xs.copy_(xh, non_blocking=True)
-        layer.linear(X_stages[0] if len(X_stages) == 1 else X_stages)
-        for yh, yd in zip(Y_hosts, Y_devs):
-            yh.copy_(yd, non_blocking=True)
+        if parts:
+            e2e_streamed(parts, X_hosts, X_stages, Y_hosts, stream, dev, a)
+        else:
+            for xs, xh in zip(X_stages, X_hosts):
+                xs.copy_(xh, non_blocking=True)
+            layer.linear(X_stages[0] if len(X_stages) == 1 else X_stages)
+            for yh, yd in zip(Y_hosts, Y_devs):
+                yh.copy_(yd, non_blocking=True)
         b.record(stream)
         torch.cuda.synchronize(dev)
         if i >= 2:
@@ -1093,7 +1153,9 @@ def main():
                        else "fgfp8_quant_static + fgfp8_gemm_rowcol") if isinstance(layer, RowColLayer)
                       else "fgfp8_linear"),
         "e2e": {"value": whole_job_rate(world, flops, r["e2e_ms"]), "unit": "TFLOP/s",
-                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"], "ms_per_step": r["e2e_ms"]},
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"], "ms_per_step": r["e2e_ms"],
+                "pipeline": (f"{E2E_CHUNKS} token chunks per layer: copy in, fgfp8_linear, copy out on three "
+                             f"streams" if streamed_parts(layer) else "copy in, the step, copy out on one stream")},
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
         "peaks": peaks,
