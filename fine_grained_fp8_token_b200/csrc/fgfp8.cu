@@ -8,6 +8,7 @@
 
 #include <cstdint>
 #include <cstdio>
+#include <map>
 #include <mutex>
 #include <set>
 #include <unordered_map>
@@ -432,9 +433,29 @@ fgfp8_status check_rows_common(const void* X, int64_t R, int64_t K, int64_t ldx,
   return FGFP8_OK;
 }
 
-unsigned grid_stride_blocks(int64_t work_items, int sm_count) {
+// CTAs of `kernel` (with `threads` threads, no dynamic shared memory) that
+// are resident on the device at once, from the occupancy calculator, cached
+// per (kernel, device).  A grid-stride kernel launched with more CTAs than
+// this runs the excess as a partial second wave that finishes last.
+int64_t resident_blocks(const void* kernel, int threads, int dev, int sm_count) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int64_t> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find({kernel, dev});
+  if (it != cache.end()) return it->second;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  const int64_t n = static_cast<int64_t>(sm_count) * per_sm;
+  cache[{kernel, dev}] = n;
+  return n;
+}
+
+// Grid of a grid-stride kernel over work_items items of one thread each:
+// enough 256-thread CTAs for the work, at most one resident wave.
+unsigned grid_stride_blocks(const void* kernel, int64_t work_items, int dev, int sm_count) {
   const int64_t want = (work_items + 255) / 256;
-  const int64_t cap = static_cast<int64_t>(sm_count) * 8;
+  const int64_t cap = resident_blocks(kernel, 256, dev, sm_count);
   return static_cast<unsigned>(want < 1 ? 1 : (want < cap ? want : cap));
 }
 
@@ -485,7 +506,11 @@ fgfp8_status quant_act_impl(const void* X, int64_t M, int64_t K, int64_t ldx, ui
   constexpr int kUnroll = 2;                 // groups in flight per 8-lane group (4 x 16-byte loads per lane)
   const uint64_t groups = static_cast<uint64_t>(M) * (K / 128);
   const uint64_t want = (groups * 8 + 256 * kUnroll - 1) / (256 * kUnroll);
-  const uint64_t cap = static_cast<uint64_t>(info.sm_count) * 8;
+  // one resident wave at most (the grid strides over the rest)
+  const uint64_t cap = static_cast<uint64_t>(
+      resident_blocks(fmt == FGFP8_SCALE_F32 ? reinterpret_cast<const void*>(fgfp8::quant_act_kernel<0, kUnroll>)
+                                             : reinterpret_cast<const void*>(fgfp8::quant_act_kernel<1, kUnroll>),
+                      256, dev, info.sm_count));
   const unsigned blocks = static_cast<unsigned>(want < cap ? (want ? want : 1) : cap);
   fgfp8::FastDiv kbd(static_cast<uint32_t>(K / 128));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -799,7 +824,9 @@ fgfp8_status fgfp8_tensor_scale(const void* X, int64_t R, int64_t K, int64_t ldx
   if (e != cudaSuccess) return cuda_fail(e, "clearing the amax word");
   if (R > 0) {
     fgfp8::FastDiv chunks(static_cast<uint32_t>(K / 8));
-    fgfp8::tensor_amax_kernel<<<grid_stride_blocks(R * (K / 8), info.sm_count), 256, 0, s>>>(
+    fgfp8::tensor_amax_kernel<<<grid_stride_blocks(reinterpret_cast<const void*>(fgfp8::tensor_amax_kernel),
+                                                   R * (K / 8), dev, info.sm_count),
+                                256, 0, s>>>(
         reinterpret_cast<const uint16_t*>(X), static_cast<uint32_t>(R), static_cast<uint32_t>(K),
         static_cast<uint64_t>(ldx), chunks, word);
     st = check_launch("tensor amax launch");
@@ -821,7 +848,9 @@ fgfp8_status fgfp8_quant_static(const void* X, int64_t R, int64_t K, int64_t ldx
   st = current_device(&dev, &info);
   if (st != FGFP8_OK) return st;
   fgfp8::FastDiv chunks(static_cast<uint32_t>(K / 8));
-  fgfp8::quant_static_kernel<<<grid_stride_blocks(R * (K / 8), info.sm_count), 256, 0,
+  fgfp8::quant_static_kernel<<<grid_stride_blocks(reinterpret_cast<const void*>(fgfp8::quant_static_kernel),
+                                                  R * (K / 8), dev, info.sm_count),
+                               256, 0,
                                reinterpret_cast<cudaStream_t>(stream)>>>(
       reinterpret_cast<const uint16_t*>(X), static_cast<uint32_t>(R), static_cast<uint32_t>(K),
       static_cast<uint64_t>(ldx), chunks, scale, Xq);
@@ -910,7 +939,9 @@ fgfp8_status fgfp8_gather_cols(const void* parts, int64_t P, int64_t M, int64_t 
   fgfp8_status st = current_device(&dev, &info);
   if (st != FGFP8_OK) return st;
   const uint32_t total = static_cast<uint32_t>(P * M * (n / 8));
-  fgfp8::gather_cols_kernel<<<grid_stride_blocks(total, info.sm_count), 256, 0,
+  fgfp8::gather_cols_kernel<<<grid_stride_blocks(reinterpret_cast<const void*>(fgfp8::gather_cols_kernel), total,
+                                                 dev, info.sm_count),
+                              256, 0,
                               reinterpret_cast<cudaStream_t>(stream)>>>(
       reinterpret_cast<const uint4*>(parts), total, fgfp8::FastDiv(static_cast<uint32_t>(n / 8)),
       fgfp8::FastDiv(static_cast<uint32_t>(M)), reinterpret_cast<uint4*>(Y));
