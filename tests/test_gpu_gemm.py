@@ -317,3 +317,32 @@ def test_grouped_linear_equals_two_calls(dev, fmt):
     Y2 = fg.grouped_linear(X, Wq, Ws, offs, fmt)
     fg.check_device_status()
     assert torch.equal(Y1, Y2)
+
+
+@pytest.mark.parametrize("fmt", [F32, UE8M0])
+@pytest.mark.parametrize("M", [7, 200])
+def test_gemm_output_beyond_bf16_range(dev, fmt, M):
+    """Outputs whose exact value lies beyond the bf16 range round to +-inf,
+    as the oracle's bf16 rounding of its fp64 result does; rows scaled down
+    to stay in range keep the GEMM tolerance.  Operands are same-signed per
+    row (|x| ~ 2^100, w ~ 2^20 up to 2^21), so no partial sum cancels: the
+    K = 512 sum reaches ~2^130 on the large rows and ~2^120 on the scaled
+    rows.  Covers the few-token kernel (M = 7) and the persistent one."""
+    N, K = 256, 512
+    g = torch.Generator().manual_seed(M + fmt)
+    mag = (1.0 + torch.rand((M, K), generator=g)) * 2.0 ** 100
+    sign = torch.where(torch.arange(M) % 2 == 0, 1.0, -1.0)[:, None]
+    rowscale = torch.where(torch.arange(M) % 3 == 2, 2.0 ** -10, 1.0)[:, None]
+    X = (mag * sign * rowscale).to(torch.bfloat16)
+    W = ((1.0 + torch.rand((N, K), generator=g)) * 2.0 ** 20).to(torch.bfloat16)
+    Y = gpu_linear(X.to(dev), W.to(dev), fmt)
+    Y_ref, S = oracle_linear(bits16(X), bits16(W), fmt)
+    Y_gpu = y_to_f64(Y)
+    ref_bits = oracle.bf16_rne(Y_ref)
+    over = np.abs(Y_ref) > 2.0 * float(np.finfo(np.float32).max)      # clearly beyond bf16 and fp32
+    finite = np.abs(Y_ref) < 0.25 * 3.3895e38                          # clearly inside
+    assert over.any() and finite.any()
+    ref_over = torch.from_numpy(ref_bits[over].astype(np.int16)).view(torch.bfloat16).double().numpy()
+    assert np.array_equal(Y_gpu[over], ref_over), "overflowing outputs differ from the oracle's bf16 rounding"
+    assert np.isinf(Y_gpu[over]).all()
+    assert_gemm_close(Y_gpu[finite], Y_ref[finite], S[finite], f"in-range rows fmt {fmt} M {M}")
