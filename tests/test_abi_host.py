@@ -186,3 +186,32 @@ def test_masked_quant_and_linear_validation():
     assert g(A, 256, A, A, 256, A, A, A, 0, 2, 128, 256, 256, 0, None) == INVALID  # NULL counts
     assert g(A, 256, A, A, 256, A, A, A, A, 2, 128, 256, 256, 3, None) == INVALID  # fmt
 
+
+
+def test_gather_cols_validation():
+    f = fg.fgfp8_gather_cols
+    assert f(A, 2, 4, 12, A, None) == SHAPE                             # n % 8
+    assert f(A, -1, 4, 16, A, None) == INVALID                          # negative
+    assert f(0, 2, 4, 16, A, None) == INVALID                           # NULL parts
+    assert f(A, 2, 4, 16, 0, None) == INVALID                           # NULL Y
+    assert f(A + 8, 2, 4, 16, A, None) == ALIGN                         # parts alignment
+    assert f(A, 2, 4, 16, A + 4, None) == ALIGN                         # Y alignment
+    assert f(A, 1 << 16, 1 << 16, 1 << 10, A, None) == SHAPE            # P * M * n / 8 >= 2^32
+    assert f(A, 0, 4, 16, A, None) == OK                                # empty: no-op
+    assert f(A, 2, 0, 16, A, None) == OK
+
+
+def test_selftest_gemm_timeout_validation():
+    f = fg.fgfp8_selftest_gemm_timeout
+    assert f(A, A, 256, A, A, A, 256, 512, 1024, 0, 8, None) == INVALID    # withhold_kb >= K/128
+    assert f(A, A, 256, A, A, A, 256, 512, 1024, 0, -1, None) == INVALID   # negative
+    assert f(A, A, 64, A, A, A, 64, 512, 1024, 0, 1, None) == SHAPE        # M <= 64: not the persistent kernel
+    assert f(A, A, 256, A, A, A, 256, 384, 1024, 0, 1, None) == SHAPE      # N % 256
+    assert f(A, A, 256, A, A, A, 256, 512, 1000, 0, 1, None) == SHAPE      # K % 128
+    assert f(A, A, 256, A, A, A, 256, 512, 1024, 3, 1, None) == INVALID    # fmt
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the behaviour without a GPU")
+def test_new_entry_points_without_gpu_fail_loudly():
+    assert fg.fgfp8_gather_cols(A, 2, 4, 16, A, None) == CUDA
+    assert fg.fgfp8_selftest_gemm_timeout(A, A, 256, A, A, A, 256, 512, 1024, 0, 1, None) == CUDA
