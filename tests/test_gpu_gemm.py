@@ -118,12 +118,15 @@ def sample_rows(M, n_random=48, seed=0):
 @pytest.mark.parametrize("cfg", [workloads.LLAMA_ATTN, workloads.LLAMA_GATE_UP, workloads.LLAMA_DOWN,
                                  *workloads.LLAMA_UE8M0.values()], ids=lambda c: c.name)
 def test_gemm_full_size_sampled_rows(dev, cfg):
+    """The full-size dense shapes the benchmark times: the first and last row
+    of every 128-row M tile plus random rows, every output column, against
+    the oracle."""
     X = workloads.activations((cfg.M, cfg.K), cfg.x_kind, cfg.seed, device=dev)
     W = workloads.weights((cfg.N, cfg.K), cfg.seed + 1, device=dev)
     Y = gpu_linear(X, W, cfg.fmt)
     rows = sample_rows(cfg.M, n_random=16 if cfg.N > 8192 else 48)
-    if cfg.N > 8192:
-        rows = rows[::2]
+    tiles = np.arange(0, cfg.M, 128)
+    assert np.isin(tiles, rows).all() and np.isin(np.minimum(tiles + 127, cfg.M - 1), rows).all()
     Y_ref, S = oracle_linear(bits16(X), bits16(W), cfg.fmt, rows=rows)
     assert_gemm_close(y_to_f64(Y[torch.as_tensor(rows, device=dev)]), Y_ref, S, cfg.name)
 
