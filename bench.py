@@ -55,6 +55,10 @@ import workloads  # noqa: E402
 
 METRIC = "block-scaled FP8 GEMM TFLOP/s (% FP8 peak); act-quant GB/s (% HBM)"
 L2_FLUSH_BYTES = 256 << 20
+# Idle time before each timed pass (the step pass and the per-kernel pass), so
+# that both start from the same power state: the per-kernel breakdown then
+# describes the step it breaks down instead of a GPU already heated by it.
+REST_S = 0.25
 FP8_OVER_BF16 = 2.0            # nominal dense fp8 / bf16 tensor ratio on B200 (4.5 / 2.25 PFLOP/s)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
@@ -160,7 +164,11 @@ class ClockSampler:
             try:
                 mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
                 reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                self.samples.append((mhz, reasons))
+                try:
+                    watts = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                except Exception:
+                    watts = None
+                self.samples.append((mhz, reasons, watts))
             except Exception:
                 pass
             self.stop_flag.wait(0.01)
@@ -185,12 +193,17 @@ class ClockSampler:
                  "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
                  "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4)}
         seen = set()
-        for _, r in self.samples:
+        for _, r, _ in self.samples:
             for n, bit in names.items():
                 if r & bit:
                     seen.add(n)
-        return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
-                "samples": len(self.samples), "reasons": sorted(seen)}
+        out = {"sm_mhz": statistics.median(m for m, _, _ in self.samples), "sm_max_mhz": self.max_mhz,
+               "samples": len(self.samples), "reasons": sorted(seen)}
+        watts = [w for _, _, w in self.samples if w is not None]
+        if watts:
+            out["power_w"] = round(statistics.median(watts), 1)
+            out["power_w_max"] = round(max(watts), 1)
+        return out
 
 
 def flush_l2(buf_w, buf_r):
@@ -822,6 +835,7 @@ def run_gpu(args, rank, world, dev):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
+    time.sleep(REST_S)
     sampler.start()
     for i in range(n):
         flush_l2(flush_w, flush_r)
@@ -836,7 +850,14 @@ def run_gpu(args, rank, world, dev):
     step_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(n)]
     total_ms = sum(step_ms)
 
-    # the kernels timed apart (same flush between steps)
+    # the kernels timed apart (same flush between steps), from the same idle
+    # start as the step pass
+    ksampler = ClockSampler(dev.index)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    time.sleep(REST_S)
+    ksampler.start()
     for i in range(n):
         flush_l2(flush_w, flush_r)
         kev[i][0].record(stream)
@@ -844,6 +865,7 @@ def run_gpu(args, rank, world, dev):
             f()
             kev[i][j + 1].record(stream)
     torch.cuda.synchronize(dev)
+    kclocks = ksampler.stop()
     layer.fg.check_device_status()
     kern_ms = [sum(kev[i][j].elapsed_time(kev[i][j + 1]) for i in range(n)) for j in range(len(kernels))]
 
@@ -893,6 +915,7 @@ def run_gpu(args, rank, world, dev):
     kernel_ms = {name: t / n for (name, _), t in zip(kernels, kern_tot)}
     return layer, {"total_ms": total_ms, "kernel_ms": kernel_ms, "gemm_ms": kernel_ms["gemm"],
                    "quant_ms": kernel_ms["quant_act"], "e2e_ms": e2e_mean, "wq_ms": wq_mean, "clocks": clocks,
+                   "clocks_kernels": kclocks,
                    "h2d": h2d, "d2h": d2h, "launches": launches_per_step * n}
 
 
@@ -1158,6 +1181,7 @@ def main():
                              f"streams" if streamed_parts(layer) else "copy in, the step, copy out on one stream")},
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
+        "clocks_kernels": r["clocks_kernels"],
         "peaks": peaks,
     }
     if hasattr(layer, "kernel_flops"):
