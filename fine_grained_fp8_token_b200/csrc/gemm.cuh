@@ -266,6 +266,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
                             int withhold_kb, int group_m) {
   using C = GemmCfg<BN, CW>;
   static_assert(!kFuse || (BN == 256 && CW == 128 && FMT == 0 && !kGrouped), "fused SwiGLU: dense fp32 256-wide");
+  static_assert(C::kStages > C::kNumBuf, "the promotion waits on the stage barriers (see the promotion loop)");
+  static_assert((2 * C::kStages + C::kNumBuf + 1 + 8) * 8 + 4 <= C::kBarrierBytes, "barrier area");
   constexpr bool kHalfTiles = !kGrouped && BN == 256 && !kFuse;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -274,8 +276,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
   uint8_t* sStg = sB + C::kStages * C::kBBytes;       // epilogue staging, one slot per promotion warp
   uint64_t* full = reinterpret_cast<uint64_t*>(sStg + C::kStagingBytes);
   uint64_t* empty = full + C::kStages;
-  uint64_t* tfull = empty + C::kStages;
-  uint64_t* tempty = tfull + C::kNumBuf;
+  uint64_t* tempty = empty + C::kStages;
   uint64_t* mma_done = tempty + C::kNumBuf;
   uint64_t* xfull = mma_done + 1;                     // fused epilogue: halves exchanged, per quadrant
   uint64_t* xempty = xfull + 4;                       // fused epilogue: half-row amax exchanged, per quadrant
@@ -326,10 +327,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < C::kNumBuf; ++b) {
-      mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], C::kEpiWarps);
-    }
+    for (int b = 0; b < C::kNumBuf; ++b) mbar_init(&tempty[b], C::kEpiWarps);
     mbar_init(mma_done, 1);
     for (int q = 0; q < 4; ++q) {
       mbar_init(&xfull[q], 64);                       // both warps of the quadrant's pair
@@ -445,8 +443,9 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
             const uint64_t bd = b_desc0 + ((s * C::kBBytes + kk * 32) >> 4);
             mma_f8f6f4(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
           }
+          // one commit per K block: the stage's "empty" barrier also tells
+          // the promotion warps that the partial of this K block is in TMEM
           mma_commit(&empty[s]);
-          mma_commit(&tfull[buf]);
         }
       }
       mma_commit(mma_done);
@@ -598,8 +597,14 @@ __global__ void __launch_bounds__(GemmCfg<BN, CW>::kThreads, 1)
           const float sc = live ? combine_raw<FMT>(ra[d], rw[d]) : 0.0f;
           fetch(kb + kScaleAhead, m, live, ws_row, ra[d], rw[d]);
           const int buf = bt % C::kNumBuf;
-          // warp-uniform outcome: the TMEM loads below are .sync.aligned
-          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[buf], (bt / C::kNumBuf) & 1u))) {
+          // The partial of K block bt is complete when the MMAs' commit to
+          // stage bt % kStages lands (phase bt / kStages of its "empty"
+          // barrier).  That barrier cannot run a phase ahead of this wait:
+          // its next phase is the commit of K block bt + kStages, whose MMAs
+          // need buffer (bt + kStages) % kNumBuf back from a later K block's
+          // promotion (kStages > kNumBuf).  Warp-uniform outcome: the TMEM
+          // loads below are .sync.aligned.
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[bt % C::kStages], (bt / C::kStages) & 1u))) {
             if (lane == 0) record_status(kDevTimeoutEpilogue);
             ok = false;
             break;
