@@ -104,14 +104,22 @@ def measured_peaks():
     return {**FALLBACK_PEAKS, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def kernel_source_sha256():
+def kernel_source_sha256(root=None):
+    """sha256 over the CUDA sources in name order: each file's name, then its
+    text with comments and blank lines removed.  A comment-only edit keeps
+    committed ncu counters valid; any change to the code invalidates them."""
     import glob
     import hashlib
+    import re
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "fine_grained_fp8_token_b200", "csrc", "*"))):
+    for f in sorted(glob.glob(os.path.join(root or ROOT, "fine_grained_fp8_token_b200", "csrc", "*"))):
         h.update(os.path.basename(f).encode())
-        with open(f, "rb") as fh:
-            h.update(fh.read())
+        with open(f, encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        code = [line.rstrip() for line in text.splitlines() if line.strip()]
+        h.update("\n".join(code).encode())
     return h.hexdigest()
 
 

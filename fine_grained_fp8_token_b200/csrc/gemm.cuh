@@ -9,8 +9,9 @@
 //               kStages shared-memory slots;
 //   warp 1      owns TMEM and issues tcgen05.mma (kind::f8f6f4, E4M3 x E4M3
 //               -> fp32), four K=32 steps per K block, into one of two TMEM
-//               partial buffers (ping-pong), then commits to the slot's
-//               "empty" barrier and the buffer's "full" barrier;
+//               partial buffers (ping-pong), then commits once to the slot's
+//               "empty" barrier, which also tells the promotion warps that
+//               the block's partial is in TMEM;
 //   warps 4..   promotion: each thread owns one output row and CW columns; it
 //               loads the block partial from TMEM, multiplies by the product
 //               of the two block scales and accumulates in fp32 registers
