@@ -19,7 +19,9 @@ __global__ void __launch_bounds__(256) gather_cols_kernel(const uint4* __restric
   const uint32_t cpr = chunks_per_row.d;                 // 16-byte chunks per part row (n / 8)
   const uint32_t M = rows.d;
   const uint32_t P_cpr = total / M;                      // chunks per output row (P * n / 8)
-  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+  const uint32_t step = gridDim.x * blockDim.x;
+  // the increment never wraps past the 32-bit count (a wrapped index would restart the pass)
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i = (total - i > step) ? i + step : total) {
     const uint32_t row = chunks_per_row.div(i);          // p * M + m
     const uint32_t c = i - row * cpr;
     const uint32_t p = rows.div(row);

@@ -175,8 +175,10 @@ __device__ __forceinline__ uint2 quant8(const uint4& v, const GroupScale& g) {
 
 // ---------------------------------------------------------------------------
 // Activation quantization.  Eight lanes per 128-element group, 16 elements
-// (two 16-byte loads) per lane, UNROLL groups in flight per lane group,
-// grid-stride over the M*K/128 groups in row-major order.
+// (two 16-byte loads) per lane, UNROLL groups in flight per lane group, over
+// the M*K/128 groups in row-major order.  The host sizes the grid to cover
+// every group in one pass where it can; the loop strides over what a capped
+// grid leaves, and never wraps past the 32-bit group count.
 // X bf16 [M, K] row stride ldx  ->  Xq u8 [M, K] row stride K,
 // scales Xs[g * ld_s + m] (fp32 or UE8M0 byte).
 // ---------------------------------------------------------------------------
@@ -193,8 +195,9 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
   const uint32_t gmask = 0xFFu << (lane & 24u);            // the 8 lanes sharing a group
   const uint32_t grp = (blockIdx.x * blockDim.x + threadIdx.x) >> 3;
   const uint32_t ngrp = (gridDim.x * blockDim.x) >> 3;
+  const uint32_t step = ngrp * UNROLL;
 
-  for (uint32_t base = grp; base < total; base += ngrp * UNROLL) {
+  for (uint32_t base = grp; base < total; base = (total - base > step) ? base + step : total) {
     uint4 v[UNROLL][2];
     uint32_t m[UNROLL], g[UNROLL];
 #pragma unroll
@@ -260,7 +263,11 @@ __global__ void __launch_bounds__(256) quant_act_masked_kernel(const uint16_t* _
   const uint32_t sub = lane & 7u;
   const uint32_t gmask = 0xFFu << (lane & 24u);
   const uint32_t row0 = e * cap;
-  for (uint32_t gi = (blockIdx.x * blockDim.x + threadIdx.x) >> 3; gi < total; gi += (gridDim.x * blockDim.x) >> 3) {
+  const uint32_t gstep = (gridDim.x * blockDim.x) >> 3;
+  // the increment never wraps past the 32-bit count (a wrapped index would
+  // restart the pass)
+  for (uint32_t gi = (blockIdx.x * blockDim.x + threadIdx.x) >> 3; gi < total;
+       gi = (total - gi > gstep) ? gi + gstep : total) {
     const uint32_t r = kb_div.div(gi);
     const uint32_t g = gi - r * kb_div.d;
     const uint32_t m = row0 + r;
@@ -430,7 +437,8 @@ __global__ void __launch_bounds__(256) tensor_amax_kernel(const uint16_t* __rest
                                                           uint32_t* __restrict__ amax_bits) {
   const uint32_t total = R * chunk_div.d;              // 16-byte chunks
   uint32_t a = 0;
-  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+  const uint32_t istep = gridDim.x * blockDim.x;
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i = (total - i > istep) ? i + istep : total) {
     const uint32_t row = chunk_div.div(i);
     const uint32_t c = i - row * chunk_div.d;
     a = max(a, absmax_bits8(ld_stream_v4(X + static_cast<uint64_t>(row) * ldx + c * 8u)));
@@ -460,7 +468,8 @@ __device__ __forceinline__ void quant_static_run(const uint16_t* __restrict__ X,
   const float r = kFast ? __frcp_rn(s) : 0.0f;
   const auto div = [s, r](float x) { return static_quotient<kFast>(fabsf(x), s, r); };
   const uint32_t total = R * chunk_div.d;
-  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+  const uint32_t istep = gridDim.x * blockDim.x;
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i = (total - i > istep) ? i + istep : total) {
     const uint32_t row = chunk_div.div(i);
     const uint32_t c = i - row * chunk_div.d;
     const uint4 v = ld_stream_v4(X + static_cast<uint64_t>(row) * ldx + c * 8u);
