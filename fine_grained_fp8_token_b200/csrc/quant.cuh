@@ -96,19 +96,6 @@ __device__ __forceinline__ GroupScale make_scale(uint32_t amax_bits) {
   return g;
 }
 
-// |x|/s for one element, x given as an fp32 (its bf16 bits in the top half).
-template <int FMT>
-__device__ __forceinline__ float quotient(float x, const GroupScale& g) {
-  const float a = fabsf(x);
-  if (FMT == 0) {
-    const float q0 = __fmul_rn(a, g.r);
-    const float e = __fmaf_rn(-q0, g.s, a);
-    return __fmaf_rn(e, g.r, q0);
-  } else {
-    return __fmul_rn(a, g.r);
-  }
-}
-
 // Four bf16 (two packed words) -> four E4M3 codes in one word (element 0 in
 // the low byte).  Magnitudes are quantized (div(x) = |x| / s); the four sign
 // bits (bit 7 of the bf16 bytes 1 and 3 of each word) are gathered with one
@@ -124,9 +111,27 @@ __device__ __forceinline__ uint32_t quant4_by(uint32_t w0, uint32_t w1, const Di
   return codes | signs;
 }
 
+// Four bf16 -> four E4M3 codes with the group's scale, in packed fp32x2
+// arithmetic (two elements per instruction).  Per element: |x| (the bf16
+// sign bit cleared before the widening), then for fp32 scales the FMA form
+// of Markstein's correctly rounded division, q0 = RN(|x| r),
+// q = RN(fma(RN(fma(-q0, s, |x|)), r, q0)) with r = RN(1/s); for UE8M0
+// scales the exact product |x| * 2^-p.  Signs and byte order as in quant4_by.
 template <int FMT>
 __device__ __forceinline__ uint32_t quant4(uint32_t w0, uint32_t w1, const GroupScale& g) {
-  return quant4_by(w0, w1, [&g](float x) { return quotient<FMT>(x, g); });
+  const float2 r2 = make_float2(g.r, g.r);
+  auto q2 = [&](uint32_t w) {
+    const float2 a = make_float2(__uint_as_float((w << 16) & 0x7FFFFFFFu), __uint_as_float(w & 0x7FFF0000u));
+    const float2 q0 = __fmul2_rn(a, r2);
+    if (FMT != 0) return q0;
+    const float2 ns2 = make_float2(-g.s, -g.s);
+    return __ffma2_rn(__ffma2_rn(q0, ns2, a), r2, q0);
+  };
+  const uint32_t c0 = __nv_cvt_float2_to_fp8x2(q2(w0), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t c1 = __nv_cvt_float2_to_fp8x2(q2(w1), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t codes = __byte_perm(c0, c1, 0x5410);
+  const uint32_t signs = __byte_perm(w0, w1, 0x7531) & 0x80808080u;
+  return codes | signs;
 }
 
 // |x| / s for a caller-given scale s > 0 (static quantization), correctly
